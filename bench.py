@@ -1,0 +1,316 @@
+"""Benchmark of the MOSS-Image DiT denoising step on B200.
+
+A bench "step" is one denoising step of the 1024^2 sampling loop: the DiT twice (CFG
+batch 2: conditional branch, unconditional branch skipping layer 22 inside the slg window
+[0.01, 1.0]), then the FP32 CFG combine and the shift-5 flow-matching Euler update.  The
+timed steps walk the 50-step schedule from step 0, so the default --steps 50 times one
+whole image.  Model: 42 blocks, hidden 3072, 24 heads of 128, FFN 8192, random N(0, 0.02)
+BF16 weights (seed 2); 512 synthetic text tokens per branch; latent noise from seed 42.
+
+Prints one JSON line (rank 0).  `value` is DiT forwards/s over all ranks (two forwards per
+step); replicas only: each rank runs its own image, no collective on the data path.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DiT forwards/s and s/image at 1024² (50 steps, CFG 3); % BF16 TC peak"
+UNIT = "forwards/s"
+HEIGHT = WIDTH = 1024
+N_TXT = 512
+STEPS_PER_IMAGE = 50
+CFG, SHIFT, SKIP, SLG = 3.0, 5.0, (22,), (0.01, 1.0)
+WORKLOAD = ("1024^2 denoising step of the 42-block DiT (hidden 3072, 24x128 heads, FFN 8192): "
+            "4096 image + 512 text tokens per branch, CFG batch 2, uncond skips layer 22 in slg [0.01, 1.0], "
+            "steps walk the 50-step shift-5 schedule")
+
+
+def flops_per_branch_layer(N, D=3072, F=8192):
+    """Algorithmic FLOPs of one block on one branch of N tokens, by kernel class."""
+    return {
+        "gemm_qkv": 2.0 * N * D * 3 * D,
+        "attention": 4.0 * N * N * D,
+        "gemm_oproj": 2.0 * N * D * D,
+        "gemm_gateup": 2.0 * N * D * 2 * F,
+        "gemm_down": 2.0 * N * F * D,
+    }
+
+
+def _slg_on(step, steps, a, b):
+    p = step / steps
+    return a <= p <= b
+
+
+def step_branch_layers(step, L=42):
+    return 2 * L - (len(SKIP) if _slg_on(step % STEPS_PER_IMAGE, STEPS_PER_IMAGE, *SLG) else 0)
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(seconds_hint=True):
+    """The oracle (float64 numpy, as it stands) on one branch-block of the 1024^2 workload:
+    4608 tokens, hidden 3072.  forwards/s = 1 / (42 * block time)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import moss_oracle as o
+    from synth import ModelShape, make_residual, make_weights, numpy_weights
+
+    shape = ModelShape(layers=1, hidden=3072, heads=24, ffn=8192)
+    wn = numpy_weights(make_weights(shape, 7))
+    x = make_residual(1, 4096 + N_TXT, 3072, 8)[0].double().numpy()
+    ang = o.rope_angles(o.token_positions(64, 64, N_TXT))
+    c = o.conditioning(0.5, wn)
+    mod = o.block_modulation(c, wn["mod_w"][0], wn["mod_b"][0])
+    lw = o.layer_weights(wn, 0)
+    t0 = time.perf_counter()
+    o.block_forward(x, lw, mod, ang, shape.heads)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": 1.0 / (42 * dt), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"one branch-block (4608 tokens x 3072, float64) timed once: {dt:.2f} s; "
+                      f"forwards/s = 1/(42 x block time)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    steps = max(1, args.steps if args.steps <= 3 else 2)
+    vals = [cpu_baseline()["value"] for _ in range(steps)]
+    cb = cpu_baseline()
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": steps, "warmup": 0, "ms_per_step": 2000.0 / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": 4096 + N_TXT, "parallelism": "none"},
+            "cpu_baseline": dict(cb, value=value),
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=STEPS_PER_IMAGE)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import diffusion_transformer_text_block_b200 as moss
+    from synth import FULL, make_text, make_weights
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    w = make_weights(FULL, 2, device="cuda")
+    model = moss.Model(FULL, w, max_tokens=4096 + N_TXT, max_batch=2, max_latent_hw=128 * 128, max_steps=50)
+    tc = make_text(1, N_TXT, FULL.hidden, 100 + rank, device="cuda")[0].contiguous()
+    tu = make_text(1, N_TXT, FULL.hidden, 200 + rank, device="cuda")[0].contiguous()
+    x = torch.empty(HEIGHT // 8, WIDTH // 8, 32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        model.denoise_step(x, tc, tu, HEIGHT, WIDTH, i % STEPS_PER_IMAGE, STEPS_PER_IMAGE, CFG, SHIFT, SKIP, *SLG)
+
+    moss.init_noise(x, 42 + rank)
+    for i in range(args.warmup):
+        step(i)
+    moss.init_noise(x, 42 + rank)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    model.profile_enable(True)
+    launches0 = moss.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    launches = moss.launch_count() - launches0
+    ms = ev0.elapsed_time(ev1)
+    prof = model.profile_read()
+    model.profile_enable(False)
+    status = moss.device_status(clear=True)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+
+    forwards = 2 * args.steps * world
+    value = forwards / (ms / 1e3)
+    ms_per_step = ms / args.steps
+
+    # roofline of the dominant kernel class (largest summed device time)
+    N = 4096 + N_TXT
+    fl = flops_per_branch_layer(N)
+    bl = sum(step_branch_layers(i) for i in range(args.steps))
+    peaks = read_peaks()
+    kernels = {}
+    for name, (n, tms) in prof.items():
+        entry = {"launches": n, "ms": round(tms, 3), "share": round(tms / ms, 4) if ms else None}
+        if name in fl and tms > 0:
+            tf = fl[name] * bl / (tms / 1e3) / 1e12
+            entry["tflops"] = round(tf, 1)
+            entry["frac"] = round(tf / peaks["bf16_tflops_sustained"], 4)
+        kernels[name] = entry
+    dom = max((k for k in fl if prof[k][1] > 0), key=lambda k: prof[k][1])
+    n_dom, ms_dom = prof[dom]
+    achieved = fl[dom] * bl / (ms_dom / 1e3) / 1e12
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops_sustained"], 4), "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 sustained",
+                "flop_per_launch": fl[dom] * bl / max(n_dom, 1)}
+    step_flops = sum(fl.values()) * bl / args.steps
+    tc_frac = step_flops * args.steps / (ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hx = torch.empty_like(x, device="cpu").pin_memory()
+        htc = tc.cpu().pin_memory()
+        htu = tu.cpu().pin_memory()
+        hx.copy_(x.cpu())
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(args.e2e_steps):
+            x.copy_(hx, non_blocking=True)
+            tc.copy_(htc, non_blocking=True)
+            tu.copy_(htu, non_blocking=True)
+            step(i)
+            hx.copy_(x, non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ems = a0.elapsed_time(a1)
+        if world > 1:
+            t = torch.tensor([ems], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": 2 * args.e2e_steps * world / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": x.numel() * 4 + tc.numel() * 4 + tu.numel() * 4,
+               "d2h_bytes_per_step": x.numel() * 4, "steps": args.e2e_steps}
+
+    model.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    cb = None if args.no_cpu_baseline or world > 1 else cpu_baseline()
+    s_per_image = ms_per_step / 1e3 * STEPS_PER_IMAGE
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": N, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: 9.9 GB of weights stream through each step"},
+        "s_per_step": round(ms_per_step / 1e3, 4),
+        "s_per_image": round(s_per_image, 3),
+        "s_per_image_note": "measured over the timed steps" if args.steps == STEPS_PER_IMAGE else
+                            "50 x mean s/step of the timed steps",
+        "tc_frac_step": round(tc_frac, 4),
+        "roofline": roofline, "kernels": kernels, "cpu_baseline": cb, "e2e": e2e,
+        "clocks": clocks.summary(), "gpu_launches": launches, "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,418 @@
+// BF16 GEMM on the sm_100a tensor cores with the DiT block's fused epilogues.
+//
+//   D[m, n] = sum_k A[m, k] * B[n, k]      A: activations [M, K], B: weights [N, K] (both
+//                                          K-contiguous, BF16), FP32 accumulation in TMEM.
+//
+// Design (one persistent CTA per SM, 192 threads, warp-specialised):
+//   warp 0      TMA producer: 128x64 A tiles and BNx64 B tiles (128-byte swizzle) into a
+//               ring of STAGES shared-memory slots, each guarded by a full/empty mbarrier.
+//   warp 1      MMA issuer: one thread issues tcgen05.mma 128xBNx16 (four per 64-wide K
+//               slice) into one of two TMEM accumulators; tcgen05.commit frees the slot
+//               and, after the last K slice, hands the accumulator to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (thread = output row), the fused
+//               element-wise tail of the op, and direct global stores.  Two accumulators
+//               let the epilogue of tile i overlap the main loop of tile i+1.
+// Tiles are visited in bands of 16 M-tiles (all N-tiles of a band before the next band),
+// so that one band of activations stays in L2 while the weights stream past it.
+//
+// Epilogues follow the block of the single-stream DiT (windpaint.ai, MOSS-Image specs:
+// 24 heads of 128, FFN 8192) with the fused tails the sibling DiT names on B200 (SGLang
+// cookbook, Qwen-Image 2.1: Lossless RoPE fusion, Lossless MLP and residual fusion,
+// Lossless Q/K normalization).
+#include "common.cuh"
+#include "internal.h"
+
+namespace moss {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kGroupM = 16;
+constexpr int kThreads = 192;
+
+template <int BN>
+struct GemmShape {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
+  const int band = tile / (kGroupM * num_n);
+  const int m0 = band * kGroupM;
+  const int bm = min(kGroupM, num_m - m0);
+  const int idx = tile - band * kGroupM * num_n;
+  mb = m0 + idx % bm;
+  nb = idx / bm;
+}
+
+__device__ __forceinline__ void store_bf16x32(bf16* dst, const uint32_t (&pk)[16]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+}
+
+// ------------------------------------------------------------------------ epilogues
+// tb: TMEM address of this warp's 32 lanes at the accumulator's first column.
+template <int BN>
+__device__ __forceinline__ void epi_f32(const EpiParams& ep, uint32_t tb, int row, int nb) {
+  for (int c = 0; c < BN / 32; ++c) {
+    const int col = nb * BN + c * 32;
+    if (col >= ep.N) break;  // warp-uniform
+    float v[32];
+    tmem_ld32f(tb + c * 32, v);
+    if (row < ep.M) {
+      float4* d = reinterpret_cast<float4*>(ep.out_f32 + static_cast<int64_t>(row) * ep.N + col);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void epi_resid(const EpiParams& ep, uint32_t tb, int row, int nb) {
+  for (int c = 0; c < BN / 32; ++c) {
+    const int col = nb * BN + c * 32;
+    if (col >= ep.N) break;
+    float v[32];
+    tmem_ld32f(tb + c * 32, v);
+    if (row < ep.M) {
+      float4* x = reinterpret_cast<float4*>(ep.out_f32 + static_cast<int64_t>(row) * ep.N + col);
+      const float4* g = reinterpret_cast<const float4*>(ep.gate + col);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 xv = x[i];
+        const float4 gv = __ldg(g + i);
+        xv.x = fmaf(gv.x, v[4 * i + 0], xv.x);
+        xv.y = fmaf(gv.y, v[4 * i + 1], xv.y);
+        xv.z = fmaf(gv.z, v[4 * i + 2], xv.z);
+        xv.w = fmaf(gv.w, v[4 * i + 3], xv.w);
+        x[i] = xv;
+      }
+    }
+  }
+}
+
+// q|k heads: x / sqrt(mean(x^2) + eps) * gain, then rotate pairs (2j, 2j+1) by the token's
+// angle j; v heads are stored unchanged.  Each 128-column head lies in one accumulator
+// half, so the thread owning a row sees the whole head.
+__device__ __forceinline__ void epi_qkv(const EpiParams& ep, uint32_t tb, int row, int nb) {
+  const int tok = row % ep.n_tok;
+  const int ld = 3 * ep.hidden;
+  for (int hh = 0; hh < 2; ++hh) {
+    const int col = nb * 256 + hh * 128;
+    if (col >= ep.N) break;
+    const int region = col / ep.hidden;  // 0 = q, 1 = k, 2 = v
+    const uint32_t th = tb + hh * 128;
+    bf16* dst = ep.out_bf16 + static_cast<int64_t>(row) * ld + col;
+    if (region < 2) {
+      float ss = 0.f;
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32f(th + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+      }
+      const float rinv = rsqrtf(ss * (1.0f / 128.0f) + ep.eps);
+      const float* gain = region == 0 ? ep.q_gain : ep.k_gain;
+      const float2* rope = ep.rope + static_cast<int64_t>(tok) * 64;
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32f(th + c * 32, v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float x0 = v[2 * i] * rinv * __ldg(gain + c * 32 + 2 * i);
+          const float x1 = v[2 * i + 1] * rinv * __ldg(gain + c * 32 + 2 * i + 1);
+          const float2 cs = __ldg(rope + c * 16 + i);
+          pk[i] = pack_bf16x2(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+        }
+        if (row < ep.M) store_bf16x32(dst + c * 32, pk);
+      }
+    } else {
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32f(th + c * 32, v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        if (row < ep.M) store_bf16x32(dst + c * 32, pk);
+      }
+    }
+  }
+}
+
+// Accumulator columns [0,128) = gate rows f0.., [128,256) = up rows f0.. of the same f.
+__device__ __forceinline__ void epi_swiglu(const EpiParams& ep, uint32_t tb, int row, int nb) {
+  const int F = ep.N;
+  for (int c = 0; c < 4; ++c) {
+    const int f = nb * 128 + c * 32;
+    if (f >= F) break;
+    float g[32], u[32];
+    tmem_ld32f(tb + c * 32, g);
+    tmem_ld32f(tb + 128 + c * 32, u);
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float a0 = g[2 * i] / (1.0f + __expf(-g[2 * i])) * u[2 * i];
+      const float a1 = g[2 * i + 1] / (1.0f + __expf(-g[2 * i + 1])) * u[2 * i + 1];
+      pk[i] = pack_bf16x2(a0, a1);
+    }
+    if (row < ep.M) store_bf16x32(ep.out_bf16 + static_cast<int64_t>(row) * F + f, pk);
+  }
+}
+
+__device__ __forceinline__ void epi_embed(const EpiParams& ep, uint32_t tb, int row, int nb) {
+  for (int c = 0; c < 8; ++c) {
+    const int col = nb * 256 + c * 32;
+    if (col >= ep.N) break;
+    float v[32];
+    tmem_ld32f(tb + c * 32, v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] += __bfloat162float(ep.bias[col + i]);
+    if (row < ep.M) {
+      for (int b = 0; b < ep.n_branch; ++b) {
+        float4* d = reinterpret_cast<float4*>(
+            ep.out_f32 + (static_cast<int64_t>(b) * ep.n_tok + row) * ep.N + col);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+    }
+  }
+}
+
+// Row = b * n_img + token; column j = (dy*2+dx)*32 + ch -> latent [b, 2r+dy, 2c+dx, ch].
+__device__ __forceinline__ void epi_out(const EpiParams& ep, uint32_t tb, int row) {
+  const int b = row / ep.n_img;
+  const int tok = row - b * ep.n_img;
+  const int r = tok / ep.grid_w;
+  const int cc = tok - r * ep.grid_w;
+  for (int c = 0; c < 4; ++c) {
+    float v[32];
+    tmem_ld32f(tb + c * 32, v);
+    if (row < ep.M) {
+      const int dy = c >> 1, dx = c & 1;
+      float4* d = reinterpret_cast<float4*>(
+          ep.out_f32 +
+          ((static_cast<int64_t>(b) * ep.lat_h8 + 2 * r + dy) * ep.lat_w8 + 2 * cc + dx) * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j = c * 32 + 4 * i;
+        d[i] = make_float4(v[4 * i] + __bfloat162float(ep.bias[j]), v[4 * i + 1] + __bfloat162float(ep.bias[j + 1]),
+                           v[4 * i + 2] + __bfloat162float(ep.bias[j + 2]),
+                           v[4 * i + 3] + __bfloat162float(ep.bias[j + 3]));
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------ the kernel
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmB2, const EpiParams ep, unsigned* err) {
+  using S = GemmShape<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S::kStages * S::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kStages * S::kStageBytes);
+  uint64_t* empty = full + S::kStages;
+  uint64_t* tfull = empty + S::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_m = (ep.M + kBM - 1) / kBM;
+  const int num_n = EPI == kEpiSwiglu ? (ep.N + 127) / 128 : (ep.N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = ep.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (EPI == kEpiSwiglu) tma_prefetch_desc(&tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int armed[S::kStages];  // parity of the last phase armed on full[s], -1 = never
+#pragma unroll
+      for (int s2 = 0; s2 < S::kStages; ++s2) armed[s2] = -1;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, mb, nb);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, err, kErrGemmProducer, abort_flag)) {
+            ok = false;
+            break;
+          }
+          armed[stage] = static_cast<int>(phase);
+          mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+          tma_load_2d(sA + stage * S::kABytes, &tmA, &full[stage], kb * kBK, mb * kBM);
+          if (EPI == kEpiSwiglu) {
+            tma_load_2d(sB + stage * S::kBBytes, &tmB, &full[stage], kb * kBK, nb * 128);
+            tma_load_2d(sB + stage * S::kBBytes + 128 * 128, &tmB2, &full[stage], kb * kBK, nb * 128);
+          } else {
+            tma_load_2d(sB + stage * S::kBBytes, &tmB, &full[stage], kb * kBK, nb * BN);
+          }
+          if (++stage == S::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the loads already issued land before the CTA can exit (bounded as well).
+        for (int s2 = 0; s2 < S::kStages; ++s2) {
+          if (armed[s2] < 0) continue;
+          const uint32_t a = smem_u32(&full[s2]);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(a, static_cast<uint32_t>(armed[s2])) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t kIdesc = idesc_bf16(kBM, BN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, err, kErrGemmMma, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, err, kErrGemmMma, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * S::kABytes);
+          const uint32_t b0 = smem_u32(sB + stage * S::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = sdesc_sw128(a0 + k * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + k * 32, 16, 1024);
+            mma_ss(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == S::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) tc_commit(&tfull[acc]);
+      }
+      // Every MMA issued by this thread has completed once `drain` flips: only then may
+      // the TMEM be released, on the normal path and after an abort alike.
+      tc_commit(drain);
+      const uint32_t a = smem_u32(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+    }
+  } else {
+    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, mb, nb);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, err, kErrGemmEpilogue, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: TMEM loads are .sync.aligned
+      tc_fence_after();
+      const int row = mb * kBM + quad * 32 + lane;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
+      if constexpr (EPI == kEpiF32) epi_f32<BN>(ep, tb, row, nb);
+      if constexpr (EPI == kEpiResid) epi_resid<BN>(ep, tb, row, nb);
+      if constexpr (EPI == kEpiQkv) epi_qkv(ep, tb, row, nb);
+      if constexpr (EPI == kEpiSwiglu) epi_swiglu(ep, tb, row, nb);
+      if constexpr (EPI == kEpiEmbed) epi_embed(ep, tb, row, nb);
+      if constexpr (EPI == kEpiOut) epi_out(ep, tb, row);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+template <int BN, int EPI>
+cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const EpiParams& ep,
+                     cudaStream_t s, unsigned* err) {
+  using S = GemmShape<BN>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         S::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int num_m = (ep.M + kBM - 1) / kBM;
+  const int num_n = EPI == kEpiSwiglu ? (ep.N + 127) / 128 : (ep.N + BN - 1) / BN;
+  const int tiles = num_m * num_n;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  if (grid <= 0) return cudaSuccess;
+  gemm_kernel<BN, EPI><<<grid, kThreads, S::kSmemBytes, s>>>(a, b, b2, ep, err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
+                        const EpiParams& ep, cudaStream_t s, unsigned* err) {
+  switch (kind) {
+    case kEpiF32: return launch_t<256, kEpiF32>(a, b, b2, ep, s, err);
+    case kEpiQkv: return launch_t<256, kEpiQkv>(a, b, b2, ep, s, err);
+    case kEpiResid: return launch_t<256, kEpiResid>(a, b, b2, ep, s, err);
+    case kEpiSwiglu: return launch_t<256, kEpiSwiglu>(a, b, b2, ep, s, err);
+    case kEpiEmbed: return launch_t<256, kEpiEmbed>(a, b, b2, ep, s, err);
+    case kEpiOut: return launch_t<128, kEpiOut>(a, b, b2, ep, s, err);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moss

@@ -1,0 +1,84 @@
+// Internal launch interface shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+namespace moss {
+
+using bf16 = __nv_bfloat16;
+
+// ------------------------------------------------------------------ GEMM epilogue kinds
+enum EpiKind : int {
+  kEpiF32 = 0,     // C = acc (FP32), test / library GEMM
+  kEpiQkv = 1,     // per-head RMSNorm + RoPE on q|k, BF16 store of q|k|v
+  kEpiResid = 2,   // x += gate * acc (FP32 read-modify-write)
+  kEpiSwiglu = 3,  // act = BF16(SiLU(acc_gate) * acc_up)
+  kEpiEmbed = 4,   // x[b, row, :] = acc + bias for every branch b
+  kEpiOut = 5,     // unpatchified velocity = acc + bias
+};
+
+struct EpiParams {
+  int M = 0, N = 0, K = 0;  // GEMM sizes; for kEpiSwiglu N = F (output width)
+  float* out_f32 = nullptr;  // kEpiF32: C [M, N]; kEpiResid/kEpiEmbed: x; kEpiOut: v
+  bf16* out_bf16 = nullptr;  // kEpiQkv: qkv [M, 3D]; kEpiSwiglu: act [M, F]
+  const float* gate = nullptr;       // kEpiResid: [N]
+  const bf16* bias = nullptr;        // kEpiEmbed, kEpiOut: [N]
+  const float* q_gain = nullptr;     // kEpiQkv: [128]
+  const float* k_gain = nullptr;     // kEpiQkv: [128]
+  const float2* rope = nullptr;      // kEpiQkv: [n_tok, 64] (cos, sin)
+  int n_tok = 0;                     // tokens per branch
+  int hidden = 0;                    // D
+  int n_branch = 0;                  // kEpiEmbed: branches written
+  int n_img = 0, grid_w = 0, lat_h8 = 0, lat_w8 = 0;  // kEpiOut
+  float eps = 1e-6f;
+};
+
+// ------------------------------------------------------------------ tensor maps
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                       uint32_t box_outer, std::string* err);
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_mid, std::string* err);
+
+int num_sms();
+
+// ------------------------------------------------------------------ kernels
+// BN = 256 for every epilogue but kEpiOut (BN = 128).  For kEpiSwiglu the B operand is two
+// maps (gate rows, up rows) of box {64, 128}; otherwise box {64, BN}.  A has box {64, 128}.
+cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
+                        const EpiParams& ep, cudaStream_t s, unsigned* err);
+constexpr int gemm_bn(EpiKind k) { return k == kEpiOut ? 128 : 256; }
+
+// qkv map: 3-D over [batch, n_tok, 3D] BF16 with box {64, 128, 1}.
+cudaError_t launch_attention(const CUtensorMap& qkv, bf16* o, int batch, int n_tok, int heads, int hidden,
+                             cudaStream_t s, unsigned* err);
+
+// rows of x (FP32, [.., D]) -> h (BF16).  With gather_n_img > 0, output row r reads x row
+// (r / gather_n_img) * gather_n_tok + r % gather_n_img (the image rows of every branch).
+cudaError_t launch_ln_mod(const float* x, const float* shift, const float* scale, bf16* h, int rows, int dim,
+                          int gather_n_img, int gather_n_tok, float eps, cudaStream_t s);
+
+bool ln_mod_supported(int dim);
+
+cudaError_t launch_cfg_euler(float* x, const float* vc, const float* vu, int64_t n, float cfg, float sigma,
+                             float sigma_next, cudaStream_t s);
+
+cudaError_t launch_noise(float* x, int64_t n, uint64_t seed, cudaStream_t s);
+
+// sc[t, :] = SiLU(W2 SiLU(W1 sinusoid(1000 ts[t]) + b1) + b2), t < T.
+cudaError_t launch_conditioning(const bf16* w1, const bf16* b1, const bf16* w2, const bf16* b2, const float* ts,
+                                float* sc, int T, int cdim, cudaStream_t s);
+
+// out[t * out_stride + r] = W[r, :] . sc[t, :] + bias[r], r < R, t < T.
+cudaError_t launch_mod_gemv(const bf16* W, const bf16* bias, const float* sc, float* out, int R, int cdim, int T,
+                            int64_t out_stride, cudaStream_t s);
+
+cudaError_t launch_rope_table(float2* table, int grid_h, int grid_w, int n_txt, cudaStream_t s);
+
+cudaError_t launch_patchify(const float* latent, bf16* tokens, int h8, int w8, cudaStream_t s);
+
+}  // namespace moss

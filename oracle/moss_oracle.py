@@ -341,6 +341,28 @@ def block_forward(x: np.ndarray, lw: dict, mod: np.ndarray, angles: np.ndarray,
     return x
 
 
+def block_forward_rows(x: np.ndarray, lw: dict, mod: np.ndarray, angles: np.ndarray, rows,
+                       heads: int, head_dim: int = 128) -> np.ndarray:
+    """The block's output for the query rows ``rows`` only: the same definition as
+    :func:`block_forward`, using that every step but attention acts row by row and that
+    attention needs the keys and values of all rows.  Returns [len(rows), D]."""
+    n, D = x.shape
+    rows = np.asarray(rows)
+    shift1, scale1, gate1, shift2, scale2, gate2 = np.split(mod, 6)
+    h = ln_modulate(x, shift1, scale1)
+    wq, wk, wv = np.split(lw["wqkv"], 3, axis=0)
+    q = (h[rows] @ wq.T).reshape(len(rows), heads, head_dim).transpose(1, 0, 2)
+    k = (h @ wk.T).reshape(n, heads, head_dim).transpose(1, 0, 2)
+    v = (h @ wv.T).reshape(n, heads, head_dim).transpose(1, 0, 2)
+    q = apply_rope(rms_norm(q, lw["q_gain"]), angles[rows])
+    k = apply_rope(rms_norm(k, lw["k_gain"]), angles)
+    o = attention(q, k, v).transpose(1, 0, 2).reshape(len(rows), D)
+    xr = x[rows] + gate1 * (o @ lw["wo"].T)
+    h2 = ln_modulate(xr, shift2, scale2)
+    a = silu(h2 @ lw["wg"].T) * (h2 @ lw["wu"].T)
+    return xr + gate2 * (a @ lw["wd"].T)
+
+
 def layer_weights(w: dict, l: int) -> dict:
     return {k: w[k][l] for k in ("wqkv", "q_gain", "k_gain", "wo", "wg", "wu", "wd")}
 

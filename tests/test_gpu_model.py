@@ -1,0 +1,154 @@
+"""Parity of the DiT block, the forward and the sampler with the oracle, through the C ABI.
+
+Bars (the method's stated tolerances): per-block relative L2 <= 1e-2 with BF16 weights
+against the float64 oracle, on the block output and on its update y - x (the residual
+alone would hide errors); the forward's velocity per branch <= 1e-2; the tiny 4-step
+sampling run >= 40 dB PSNR against the oracle's.
+"""
+import numpy as np
+import pytest
+import torch
+
+import diffusion_transformer_text_block_b200 as moss
+from oracle import moss_oracle as o
+from synth import TINY, make_latent, make_residual, make_text
+from tests.gpu_common import WIDE1, assert_no_device_error, make_model, psnr, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _block_case(shape, seed, gh, gw, n_txt, batch, t, layer=0, layers=None):
+    N = gh * gw + n_txt
+    model, wg, wn = make_model(shape, seed, max_tokens=N, max_batch=batch, max_latent_hw=4 * gh * gw,
+                               layers=layers)
+    x = make_residual(batch, N, shape.hidden, seed + 1)
+    xg = x.cuda()
+    model.block_forward(layer, xg, gh, gw, n_txt, t)
+    torch.cuda.synchronize()
+    y = xg.cpu().double().numpy()
+    c = o.conditioning(t, wn)
+    mod = o.block_modulation(c, wn["mod_w"][layer], wn["mod_b"][layer])
+    ang = o.rope_angles(o.token_positions(gh, gw, n_txt))
+    lw = o.layer_weights(wn, layer)
+    return model, x.double().numpy(), y, lw, mod, ang
+
+
+@pytest.mark.parametrize("gh,gw,n_txt,batch", [(4, 4, 16, 2), (8, 10, 60, 2), (2, 3, 0, 1), (1, 1, 300, 2)])
+def test_block_tiny(gh, gw, n_txt, batch):
+    model, x, y, lw, mod, ang = _block_case(TINY, 31, gh, gw, n_txt, batch, 0.5, layer=1)
+    for b in range(batch):
+        ref = o.block_forward(x[b], lw, mod, ang, TINY.heads)
+        assert rel_l2(y[b], ref) <= 1e-2
+        assert rel_l2(y[b] - x[b], ref - x[b]) <= 1e-2, rel_l2(y[b] - x[b], ref - x[b])
+    model.close()
+    assert_no_device_error()
+
+
+def test_block_full_width_one_block():
+    """One full-width block: 256x256 image (256 image tokens) + 128 text tokens, batch 2,
+    t = 0.5, FP32 residual stream."""
+    model, x, y, lw, mod, ang = _block_case(WIDE1, 41, 16, 16, 128, 2, 0.5)
+    for b in range(2):
+        ref = o.block_forward(x[b], lw, mod, ang, WIDE1.heads)
+        assert rel_l2(y[b], ref) <= 1e-2
+        assert rel_l2(y[b] - x[b], ref - x[b]) <= 1e-2, rel_l2(y[b] - x[b], ref - x[b])
+    model.close()
+    assert_no_device_error()
+
+
+def test_block_full_size_sampled_rows():
+    """The 1024^2 block shape the benchmark times (4096 image + 512 text tokens, batch 2):
+    sampled rows against the oracle's row-restricted block."""
+    gh = gw = 64
+    n_txt = 512
+    model, x, y, lw, mod, ang = _block_case(WIDE1, 43, gh, gw, n_txt, 2, 0.83)
+    N = gh * gw + n_txt
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 1, 63, 64, 4095, 4096, N - 1], rng.integers(0, N, 25)]))
+    for b in range(2):
+        ref = o.block_forward_rows(x[b], lw, mod, ang, rows, WIDE1.heads)
+        assert rel_l2(y[b][rows], ref) <= 1e-2
+        assert rel_l2(y[b][rows] - x[b][rows], ref - x[b][rows]) <= 1e-2
+    model.close()
+    assert_no_device_error()
+
+
+def test_forward_tiny_with_uncond_skip():
+    model, wg, wn = make_model(TINY, 51, max_tokens=32, max_latent_hw=64)
+    lat = make_latent(8, 8, 52)
+    txt = make_text(2, 16, TINY.hidden, 53)
+    v = model.forward(lat.cuda(), txt.cuda(), 64, 64, 0.3, skip_layers=[[], [1]])
+    torch.cuda.synchronize()
+    ref = o.dit_forward(lat.numpy(), txt.double().numpy(), 0.3, [(), (1,)], wn, TINY.heads)
+    got = v.cpu().double().numpy()
+    for b in range(2):
+        assert rel_l2(got[b], ref[b]) <= 1e-2, rel_l2(got[b], ref[b])
+    # the skipped branch really differs from an unskipped one
+    v2 = model.forward(lat.cuda(), txt.cuda(), 64, 64, 0.3, skip_layers=[[], []])
+    assert rel_l2(v2.cpu().numpy()[1], got[1]) > 1e-3
+    model.close()
+    assert_no_device_error()
+
+
+def test_forward_tiny_skip_all_layers():
+    model, wg, wn = make_model(TINY, 55, max_tokens=48, max_latent_hw=4 * 4 * 8 * 4)
+    lat = make_latent(8, 16, 56)  # 64 x 128 image: 32 image tokens
+    txt = make_text(1, 16, TINY.hidden, 57)
+    v = model.forward(lat.cuda(), txt.cuda(), 64, 128, 0.9, skip_layers=[[0, 1]])
+    ref = o.dit_forward(lat.numpy(), txt.double().numpy(), 0.9, [(0, 1)], wn, TINY.heads)
+    assert rel_l2(v.cpu().numpy()[0], ref[0]) <= 1e-2
+    model.close()
+    assert_no_device_error()
+
+
+def test_sample_tiny_psnr():
+    """The tiny sampling run: 64x64 image, 4 flow-Euler steps, shift 5, CFG 3, uncond skips
+    block 1 inside [0.01, 1.0], seed 0."""
+    model, wg, wn = make_model(TINY, 61, max_tokens=32, max_latent_hw=64, max_steps=4)
+    tc = make_text(1, 16, TINY.hidden, 62)[0]
+    tu = make_text(1, 16, TINY.hidden, 63)[0]
+    out = model.sample(tc.cuda(), tu.cuda(), 64, 64, steps=4, cfg=3.0, shift=5.0, seed=0,
+                       uncond_skip_layers=[1], slg_start=0.01, slg_stop=1.0)
+    torch.cuda.synchronize()
+    ref = o.sample(wn, TINY.heads, 64, 64, tc.double().numpy(), tu.double().numpy(), steps=4, cfg=3.0, shift=5.0,
+                   seed=0, uncond_skip_layers=(1,), slg_start=0.01, slg_stop=1.0)
+    p = psnr(ref, out.cpu().numpy())
+    assert p >= 40.0, p
+    model.close()
+    assert_no_device_error()
+
+
+def test_denoise_step_cfg1_and_sample_consistency():
+    model, wg, wn = make_model(TINY, 71, max_tokens=32, max_latent_hw=64, max_steps=4)
+    tc = make_text(1, 16, TINY.hidden, 72)[0].cuda()
+    tu = make_text(1, 16, TINY.hidden, 73)[0].cuda()
+    # sample == noise + the same denoising steps called one by one (bitwise)
+    a = model.sample(tc, tu, 64, 64, steps=3, seed=5, uncond_skip_layers=[1])
+    x = torch.empty(8, 8, 32, device="cuda")
+    moss.init_noise(x, 5)
+    for i in range(3):
+        model.denoise_step(x, tc, tu, 64, 64, i, 3, uncond_skip_layers=[1])
+    assert torch.equal(a, x)
+    # CFG 1 runs no unconditional pass: NaN negative text cannot reach the result
+    bad = torch.full_like(tu, float("nan"))
+    y = model.sample(tc, bad, 64, 64, steps=2, cfg=1.0, seed=5)
+    assert torch.isfinite(y).all()
+    ref = o.sample(wn, TINY.heads, 64, 64, tc.cpu().double().numpy(), None, steps=2, cfg=1.0, seed=5)
+    assert psnr(ref, y.cpu().numpy()) >= 40.0
+    model.close()
+    assert_no_device_error()
+
+
+def test_invalid_requests_launch_nothing():
+    model, wg, wn = make_model(TINY, 81, max_tokens=32, max_latent_hw=64)
+    lat = torch.zeros(8, 8, 32, device="cuda")
+    txt = torch.zeros(2, 16, TINY.hidden, device="cuda")
+    before = moss.launch_count()
+    with pytest.raises(moss.MossError, match="multiples of 16"):
+        model.forward(lat, txt, 60, 64, 0.5)
+    with pytest.raises(moss.MossError, match="out of range"):
+        model.forward(lat, txt, 64, 64, 0.5, skip_layers=[[], [2]])
+    with pytest.raises(moss.MossError, match="max_tokens"):
+        model.forward(lat, torch.zeros(2, 17, TINY.hidden, device="cuda"), 64, 64, 0.5)
+    assert moss.launch_count() == before
+    model.close()

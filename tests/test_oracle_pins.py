@@ -432,3 +432,12 @@ def test_psnr():
     ref = np.array([0.0, 1.0, 2.0, 3.0])
     assert o.psnr(ref, ref) == float("inf")
     assert abs(o.psnr(ref, ref + 0.03) - 10 * math.log10(9 / 0.0009)) < 1e-9
+
+
+def test_block_rows_equals_full_block():
+    w, ang, x, mod = _tiny_setup()
+    lw = o.layer_weights(w, 0)
+    full = o.block_forward(x, lw, mod, ang, TINY.heads)
+    rows = [0, 5, 17, 31]
+    np.testing.assert_allclose(o.block_forward_rows(x, lw, mod, ang, rows, TINY.heads), full[rows],
+                               rtol=1e-12, atol=1e-12)
