@@ -85,11 +85,15 @@ def test_cfg_euler(n):
     dt = abs(np.float32(s1) - np.float32(s0))
     scale = np.abs(x.numpy()) + dt * (np.abs(vu.numpy()) + 3.0 * (np.abs(vc.numpy()) + np.abs(vu.numpy())))
     assert np.all(np.abs(xg.cpu().numpy() - ref) <= 1e-6 * scale)
-    # the special cases of the pages: cfg = 1 -> v_c; v_c = v_u -> that velocity
+    # cfg = 1 -> the conditional velocity, up to the rounding of v_u + (v_c - v_u)
     x1 = x.cuda()
     moss.cfg_euler_step(x1, vc.cuda(), vu.cuda(), 1.0, s0, s1)
     ref1 = o.euler_update(x.numpy(), vc.numpy(), s0, s1)
-    assert np.all(np.abs(x1.cpu().numpy() - ref1) <= 1e-6 * (np.abs(x.numpy()) + dt * np.abs(vc.numpy())))
+    assert np.all(np.abs(x1.cpu().numpy() - ref1) <= 1e-6 * scale)
+    # v_u = v_c (what the step passes when no negative branch runs): exactly x + dt v_c
+    x2 = x.cuda()
+    moss.cfg_euler_step(x2, vc.cuda(), vc.cuda(), 1.0, s0, s1)
+    assert np.all(np.abs(x2.cpu().numpy() - ref1) <= 1e-6 * (np.abs(x.numpy()) + dt * np.abs(vc.numpy())))
 
 
 @pytest.mark.parametrize("n,seed", [(4, 0), (1001, 42), (128 * 128 * 32, 42), (64, (1 << 40) + 3)])
