@@ -167,6 +167,61 @@ def run_reference(args):
     return 0
 
 
+def run_op(args):
+    """Kernel-level timing on the 1024^2 shapes (batch 2, 4096 image + 512 text tokens):
+    `block` runs one full-width block (hidden 3072, 24x128 heads, FFN 8192) in place,
+    `attention` the attention kernel alone.  Prints one JSON line of per-class device time.
+    Used for ncu captures of single kernels on a small, one-layer case."""
+    import torch
+
+    import diffusion_transformer_text_block_b200 as moss
+    from synth import ModelShape, make_residual, make_weights
+
+    shape = ModelShape(layers=1, hidden=3072, heads=24, ffn=8192)
+    N = 4096 + N_TXT
+    if args.op == "attention":
+        g = torch.Generator(device="cuda").manual_seed(5)
+        qkv = torch.randn(2, N, 3 * 3072, generator=g, device="cuda").to(torch.bfloat16)
+        for _ in range(args.warmup):
+            moss.op_attention(qkv, 24)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            moss.op_attention(qkv, 24)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        tf = 2 * flops_per_branch_layer(N)["attention"] / (ms / 1e3) / 1e12
+        print(json.dumps({"op": "attention", "ms": round(ms, 4), "tflops": round(tf, 1)}), flush=True)
+        return 0
+    w = {k: v for k, v in make_weights(shape, 3, device="cuda").items()}
+    model = moss.Model(shape, w, max_tokens=N, max_batch=2, max_latent_hw=128 * 128, max_steps=1)
+    x = make_residual(2, N, 3072, 4, device="cuda")
+    for _ in range(args.warmup):
+        model.block_forward(0, x, 64, 64, N_TXT, 0.5)
+    torch.cuda.synchronize()
+    model.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        model.block_forward(0, x, 64, 64, N_TXT, 0.5)
+    e1.record()
+    torch.cuda.synchronize()
+    prof = model.profile_read()
+    fl = flops_per_branch_layer(N)
+    out = {"op": "block", "ms_per_block": round(e0.elapsed_time(e1) / args.steps, 4)}
+    for k, (n, tms) in prof.items():
+        if n:
+            out[k] = {"ms": round(tms / n, 4)}
+            if k in fl:
+                out[k]["tflops"] = round(2 * fl[k] / (tms / n / 1e3) / 1e12, 1)
+    out["device_status"] = moss.device_status(clear=True)
+    model.close()
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -175,9 +230,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["block", "attention"], default=None,
+                    help="time one kernel class on the 1024^2 shapes instead of the denoising step")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op:
+        return run_op(args)
 
     import torch
     import torch.distributed as dist

@@ -74,7 +74,11 @@ _SIGS = {
     "moss_op_attention": (_I, [_P, _P, _I, _I, _I, _P]),
     "moss_op_ln_modulate": (_I, [_P, _P, _P, _P, _I, _I, _P]),
     "moss_op_modulation": (_I, [_P, _F, _P, _P]),
+    "moss_modulation_noalloc": (_I, [ctypes.POINTER(Config), ctypes.POINTER(Weights), ctypes.POINTER(_F), _I, _P,
+                                     _P]),
 }
+
+NOALLOC_MAX_TIMESTEPS = 64
 
 
 def lib():
@@ -188,6 +192,35 @@ def op_ln_modulate(x, shift, scale, stream=None):
     _check(lib().moss_op_ln_modulate(_ptr(x, f, "x"), _ptr(shift, f, "shift"), _ptr(scale, f, "scale"),
                                      h.data_ptr(), rows, dim, _stream(stream)))
     return h
+
+
+def _config_for(shape, layers: int) -> Config:
+    cfg = Config()
+    lib().moss_config_init(ctypes.byref(cfg), ctypes.sizeof(Config))
+    cfg.layers, cfg.hidden, cfg.heads, cfg.head_dim = layers, shape.hidden, shape.heads, shape.head_dim
+    cfg.ffn, cfg.cond_dim = shape.ffn, shape.c_t
+    return cfg
+
+
+def modulation_noalloc(shape, weights: dict, ts: Sequence[float], out=None, stream=None):
+    """Modulation vectors for the timesteps `ts` through the allocation-free entry point:
+    returns (or fills) a CUDA FP32 tensor [len(ts), L*6D + 2D].  Only `out` is allocated
+    here (by torch, when not given); the library itself allocates nothing."""
+    import torch
+    L = weights["mod_w"].shape[0]
+    D = shape.hidden
+    if out is None:
+        out = torch.empty(len(ts), L * 6 * D + 2 * D, device="cuda", dtype=torch.float32)
+    cfg = _config_for(shape, L)
+    w = Weights()
+    lib().moss_weights_init(ctypes.byref(w), ctypes.sizeof(Weights))
+    for name in WEIGHT_FIELDS:
+        want = torch.float32 if name in ("q_gain", "k_gain") else torch.bfloat16
+        setattr(w, name, _ptr(weights[name], want, name))
+    tarr = (ctypes.c_float * max(len(ts), 1))(*ts)
+    _check(lib().moss_modulation_noalloc(ctypes.byref(cfg), ctypes.byref(w), tarr, len(ts),
+                                         _ptr(out, torch.float32, "out"), _stream(stream)))
+    return out
 
 
 def _skip_array(skips: Sequence[Sequence[int]]):

@@ -45,6 +45,13 @@ static int cuda_fail(cudaError_t e, const char* what) {
 
 static std::atomic<int64_t> g_launches{0};
 
+int set_error(int code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+
+void count_launches(int n) { g_launches += n; }
+
 // ------------------------------------------------------------------------------ device info
 int num_sms() {
   static int cached[64] = {0};

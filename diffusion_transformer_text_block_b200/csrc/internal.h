@@ -46,6 +46,11 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint6
 
 int num_sms();
 
+// Record `msg` as the calling thread's last error (cleared for MOSS_OK) and return `code`.
+int set_error(int code, const std::string& msg);
+// Add n kernel launches to the library's launch counter.
+void count_launches(int n);
+
 // ------------------------------------------------------------------ kernels
 // BN = 256 for every epilogue but kEpiOut (BN = 128).  For kEpiSwiglu the B operand is two
 // maps (gate rows, up rows) of box {64, 128}; otherwise box {64, BN}.  A has box {64, 128}.

@@ -256,6 +256,36 @@ int moss_op_ln_modulate(const float* x, const float* shift, const float* scale, 
  * layers and of the final layer, mod device FP32 [L*6D + 2D]. */
 int moss_op_modulation(moss_model* m, float t, float* mod, void* stream);
 
+/* ------------------------------------------------------------------------------------ */
+/* Allocation-free entry point.                                                          */
+/* ------------------------------------------------------------------------------------ */
+
+/* Limits of the fixed scratch used by moss_modulation_noalloc. */
+#define MOSS_NOALLOC_MAX_TIMESTEPS 64
+#define MOSS_NOALLOC_MAX_COND_DIM 256
+
+/* The modulation vectors of moss_op_modulation (all layers, then the final layer) for n_t
+ * timesteps, computed without allocating any memory and without a moss_model.  The pages
+ * have no counterpart: this exists for callers that must not allocate device memory, such
+ * as a serving process whose memory is reserved up front by its own allocator (a cudaMalloc
+ * there fails or fragments the reserve), or a latency-critical thread that cannot afford the
+ * implicit device synchronisation cudaMalloc may perform.
+ *   cfg, w:   model shape and weights as for moss_model_create; only t_w1, t_b1, t_w2, t_b2,
+ *             mod_w, mod_b, final_mod_w and final_mod_b are read.
+ *   t_host:   host float [n_t], the timesteps (sigma); 1 <= n_t <= MOSS_NOALLOC_MAX_TIMESTEPS.
+ *   mod_out:  device FP32 [n_t, L*6D + 2D], caller-owned, 16-byte aligned.
+ * Scratch: the timesteps and the n_t conditioning vectors (at most 64 x 256 floats) live in
+ * one fixed array in device memory (64 KB + 256 B) that the library reserves on every GPU it
+ * is loaded on, for the life of the process.  The first call on a device looks up that
+ * array's device address (once per device); make that first call before any stream capture.
+ * Every call uses the same array: two calls whose work overlaps on the GPU (on different
+ * streams, or from different threads) race on it, so serialise them.  Each call overwrites
+ * all the scratch it reads, so results never depend on an earlier call.
+ * Errors: INVALID_ARGUMENT (NULL or misaligned pointer, n_t or cond_dim beyond the limits
+ * above), ABI_MISMATCH (struct_size), CUDA.  Calls no allocation routine. */
+int moss_modulation_noalloc(const moss_config* cfg, const moss_weights* w, const float* t_host, int n_t,
+                            float* mod_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
