@@ -302,10 +302,9 @@ int block_impl(moss_model* m, int l, float* x, int nb, int N, const float* mod_l
   const int D = c.hidden, F = c.ffn, H = c.heads;
   const int M = nb * N;
   std::string e;
-  CUtensorMap tm_h, tm_attn, tm_act, tm_qkv3;
+  CUtensorMap tm_h, tm_attn, tm_act;
   if (!make_tmap_bf16_2d(&tm_h, m->h, D, M, 64, 128, &e) || !make_tmap_bf16_2d(&tm_attn, m->attn, D, M, 64, 128, &e) ||
-      !make_tmap_bf16_2d(&tm_act, m->act, F, M, 64, 128, &e) ||
-      !make_tmap_bf16_3d(&tm_qkv3, m->qkv, 3 * D, N, nb, 64, 128, &e))
+      !make_tmap_bf16_2d(&tm_act, m->act, F, M, 64, 128, &e))
     return fail(MOSS_ERR_CUDA, e);
 
   LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(x, mod_l, mod_l + D, m->h, M, D, 0, 0, 1e-6f, s), "ln_modulate 1");
@@ -318,7 +317,8 @@ int block_impl(moss_model* m, int l, float* x, int nb, int N, const float* mod_l
   q.rope = m->rope; q.n_tok = N; q.hidden = D;
   LAUNCH(m, MOSS_K_GEMM_QKV, s, launch_gemm(kEpiQkv, tm_h, m->tm_qkv[l], m->tm_qkv[l], q, s, m->err), "qkv gemm");
 
-  LAUNCH(m, MOSS_K_ATTENTION, s, launch_attention(tm_qkv3, m->attn, nb, N, H, D, s, m->err), "attention");
+  LAUNCH(m, MOSS_K_ATTENTION, s, launch_attention(m->qkv, m->attn, nb, N, H, D, s, m->err, &e),
+         e.empty() ? "attention" : e.c_str());
 
   EpiParams o;
   o.M = M; o.N = D; o.K = D;
@@ -790,11 +790,10 @@ int moss_op_attention(const void* qkv, void* o, int batch, int n_tok, int heads,
   if (!err) return fail(MOSS_ERR_CUDA, "device error word");
   const int D = heads * 128;
   std::string e;
-  CUtensorMap tm;
-  if (!make_tmap_bf16_3d(&tm, qkv, 3 * D, n_tok, batch, 64, 128, &e)) return fail(MOSS_ERR_CUDA, e);
   ++g_launches;
-  cudaError_t ce = launch_attention(tm, static_cast<bf16*>(o), batch, n_tok, heads, D, static_cast<cudaStream_t>(stream), err);
-  return ce == cudaSuccess ? MOSS_OK : cuda_fail(ce, "attention");
+  cudaError_t ce = launch_attention(static_cast<const bf16*>(qkv), static_cast<bf16*>(o), batch, n_tok, heads, D,
+                                    static_cast<cudaStream_t>(stream), err, &e);
+  return ce == cudaSuccess ? MOSS_OK : cuda_fail(ce, e.empty() ? "attention" : e.c_str());
 }
 
 int moss_op_ln_modulate(const float* x, const float* shift, const float* scale, void* h, int rows, int dim,

@@ -5,17 +5,19 @@
 // (MossInfer integration guide, What works: exact attention; windpaint.ai MOSS-Image specs:
 // 24 heads of 128, image and text tokens in one sequence.)
 //
-// One CTA per (128-query tile, head, branch); two CTAs share an SM so that one CTA's
-// softmax overlaps the other's matrix products.  Per CTA (192 threads):
-//   warp 0      TMA: the Q tile once, then K_j and V_j (128 keys x 128 dims each, two
-//               64-column boxes with 128-byte swizzle) for j = 0.. in order.
-//   warp 1      one thread issues S = Q K_j^T (tcgen05, both operands from shared memory,
-//               result FP32 in TMEM columns [0,128)) and O += P V_j (P from TMEM, V from
-//               shared memory as an MN-major operand, O in TMEM columns [128,256)).
-//   warps 2..5  softmax, one query row per thread: online softmax in the log2 domain,
-//               P written back as BF16 over the first 64 columns of S, and the lazy
-//               rescale of O (only when the running maximum grows by more than 2^8).
-//               At the end O / l is stored as BF16.
+// One CTA per (128-query tile, head, branch); two CTAs share an SM.  Keys are taken 64 at a
+// time.  TMEM (256 columns per CTA): S buffers 0 and 1 (64 columns each, FP32) and O (128).
+// Per CTA (192 threads):
+//   warp 0      TMA: the Q tile once, then K_j and V_j (64 keys x 128 dims, two 64-column
+//               boxes with 128-byte swizzle) into two-slot rings.
+//   warp 1      one thread issues, in this order, S_0, S_1, PV_0, S_2, PV_1, ...:
+//               S_j = Q K_j^T into S buffer j%2 (operands in shared memory) and
+//               O += P_j V_j (P_j from TMEM, V_j from shared memory as an MN-major operand).
+//               S_j+1 is computed while the softmax warps work on S_j.
+//   warps 2..5  softmax, one query row per thread: online softmax in the log2 domain, P_j as
+//               BF16 over the first 32 columns of its S buffer, lazy rescale of O (only when
+//               the running maximum grows by more than 2^8, after waiting for the PV product
+//               in flight).  At the end O / l is stored as BF16.
 // Keys past the sequence end (the TMA fills them with zeros) are masked to -inf.
 #include "common.cuh"
 #include "internal.h"
@@ -25,10 +27,12 @@ namespace moss {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kTile = 128;               // queries per CTA and keys per step
-constexpr int kHalfBytes = kTile * 128;  // one 64-column (128-byte) box of 128 rows
-constexpr int kTileBytes = 2 * kHalfBytes;
-constexpr int kSmemBytes = 3 * kTileBytes + 1024 + 256;
+constexpr int kQTile = 128;                     // queries per CTA
+constexpr int kKTile = 64;                      // keys per step
+constexpr int kBox = 64 * 128;                  // one TMA box: 64 rows x 64 BF16 columns
+constexpr int kQBytes = 4 * kBox;               // Q: 128 rows x 128 dims
+constexpr int kKVBytes = 2 * kBox;              // K_j or V_j: 64 rows x 128 dims
+constexpr int kSmemBytes = kQBytes + 4 * kKVBytes + 1024 + 256;
 constexpr uint32_t kTmemCols = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -37,37 +41,40 @@ __global__ void __launch_bounds__(kThreads, 2)
                 float scale_log2, unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Q halves (dims 0..63, 64..127) are 128 rows x 128 B each: rows 0..63 then 64..127.
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTileBytes;
-  uint8_t* sV = smem + 2 * kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 3 * kTileBytes);
+  uint8_t* sK = smem + kQBytes;                  // 2 slots
+  uint8_t* sV = smem + kQBytes + 2 * kKVBytes;   // 2 slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kQBytes + 4 * kKVBytes);
   uint64_t* b_q = bars + 0;
-  uint64_t* b_kfull = bars + 1;
-  uint64_t* b_kempty = bars + 2;
-  uint64_t* b_vfull = bars + 3;
-  uint64_t* b_vempty = bars + 4;
-  uint64_t* b_s = bars + 5;
-  uint64_t* b_p = bars + 6;
-  uint64_t* b_o = bars + 7;
-  uint64_t* b_drain = bars + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  uint64_t* b_kfull = bars + 1;   // [2]
+  uint64_t* b_kempty = bars + 3;  // [2]
+  uint64_t* b_vfull = bars + 5;   // [2]
+  uint64_t* b_vempty = bars + 7;  // [2]
+  uint64_t* b_s = bars + 9;       // [2] S_j complete, per S buffer
+  uint64_t* b_p = bars + 11;      // [2] P_j written, per S buffer
+  uint64_t* b_o = bars + 13;      // PV_j complete (one phase per j)
+  uint64_t* b_drain = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * kTile;
+  const int q0 = blockIdx.x * kQTile;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
-  const int nkv = (n_tok + kTile - 1) / kTile;
+  const int nkv = (n_tok + kKTile - 1) / kKTile;
 
   if (threadIdx.x == 0) {
     mbar_init(b_q, 1);
-    mbar_init(b_kfull, 1);
-    mbar_init(b_kempty, 1);
-    mbar_init(b_vfull, 1);
-    mbar_init(b_vempty, 1);
-    mbar_init(b_s, 1);
-    mbar_init(b_p, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b_kfull[i], 1);
+      mbar_init(&b_kempty[i], 1);
+      mbar_init(&b_vfull[i], 1);
+      mbar_init(&b_vempty[i], 1);
+      mbar_init(&b_s[i], 1);
+      mbar_init(&b_p[i], 4);
+    }
     mbar_init(b_o, 1);
     mbar_init(b_drain, 1);
     *abort_flag = 0;
@@ -82,75 +89,88 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;        // S (FP32) and P (BF16 pairs in the first 64 columns)
-  const uint32_t tO = tmem + 128;  // O (FP32)
+  const uint32_t tO = tmem + 128;  // O (FP32); S buffer i at tmem + 64 i
 
   if (warp == 0) {
     if (lane == 0) {
       const int xq = h * 128, xk = hidden + h * 128, xv = 2 * hidden + h * 128;
-      int k_armed = -1, v_armed = -1;  // parity of the last armed phase
-      bool ok = true;
-      mbar_arrive_expect_tx(b_q, kTileBytes);
-      tma_load_3d(sQ, &tm, b_q, xq, q0, b);
-      tma_load_3d(sQ + kHalfBytes, &tm, b_q, xq + 64, q0, b);
-      for (int j = 0; j < nkv && ok; ++j) {
-        if (j > 0 && !mbar_wait(b_kempty, (j - 1) & 1, err, kErrAttnProducer, abort_flag)) {
-          ok = false;
-          break;
-        }
-        k_armed = j & 1;
-        mbar_arrive_expect_tx(b_kfull, kTileBytes);
-        tma_load_3d(sK, &tm, b_kfull, xk, j * kTile, b);
-        tma_load_3d(sK + kHalfBytes, &tm, b_kfull, xk + 64, j * kTile, b);
-        if (j > 0 && !mbar_wait(b_vempty, (j - 1) & 1, err, kErrAttnProducer, abort_flag)) {
-          ok = false;
-          break;
-        }
-        v_armed = j & 1;
-        mbar_arrive_expect_tx(b_vfull, kTileBytes);
-        tma_load_3d(sV, &tm, b_vfull, xv, j * kTile, b);
-        tma_load_3d(sV + kHalfBytes, &tm, b_vfull, xv + 64, j * kTile, b);
+      int k_armed[2] = {-1, -1}, v_armed[2] = {-1, -1};  // parity of the last armed phase
+      mbar_arrive_expect_tx(b_q, kQBytes);
+      for (int half = 0; half < 2; ++half)
+        for (int r = 0; r < 2; ++r)
+          tma_load_3d(sQ + half * 2 * kBox + r * kBox, &tm, b_q, xq + 64 * half, q0 + 64 * r, b);
+      for (int j = 0; j < nkv; ++j) {
+        const int slot = j & 1;
+        const uint32_t use = (j >> 1) & 1;  // this slot's use count parity
+        if (j >= 2 && !mbar_wait(&b_kempty[slot], use ^ 1, err, kErrAttnProducer, abort_flag)) break;
+        k_armed[slot] = static_cast<int>(use);
+        mbar_arrive_expect_tx(&b_kfull[slot], kKVBytes);
+        tma_load_3d(sK + slot * kKVBytes, &tm, &b_kfull[slot], xk, j * kKTile, b);
+        tma_load_3d(sK + slot * kKVBytes + kBox, &tm, &b_kfull[slot], xk + 64, j * kKTile, b);
+        if (j >= 2 && !mbar_wait(&b_vempty[slot], use ^ 1, err, kErrAttnProducer, abort_flag)) break;
+        v_armed[slot] = static_cast<int>(use);
+        mbar_arrive_expect_tx(&b_vfull[slot], kKVBytes);
+        tma_load_3d(sV + slot * kKVBytes, &tm, &b_vfull[slot], xv, j * kKTile, b);
+        tma_load_3d(sV + slot * kKVBytes + kBox, &tm, &b_vfull[slot], xv + 64, j * kKTile, b);
       }
       // Before the CTA may exit, every load issued must have landed (bounded wait).
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(smem_u32(b_q), 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
-      if (k_armed >= 0)
-        while (!mbar_try_wait(smem_u32(b_kfull), k_armed) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
-        }
-      if (v_armed >= 0)
-        while (!mbar_try_wait(smem_u32(b_vfull), v_armed) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
-        }
+      for (int i = 0; i < 2; ++i) {
+        if (k_armed[i] >= 0)
+          while (!mbar_try_wait(smem_u32(&b_kfull[i]), k_armed[i]) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        if (v_armed[i] >= 0)
+          while (!mbar_try_wait(smem_u32(&b_vfull[i]), v_armed[i]) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+          }
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16(128, 128, false);
+      constexpr uint32_t kIdescS = idesc_bf16(128, kKTile, false);
       constexpr uint32_t kIdescO = idesc_bf16(128, 128, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       bool ok = mbar_wait(b_q, 0, err, kErrAttnMma, abort_flag);
-      for (int j = 0; j < nkv && ok; ++j) {
-        if (!mbar_wait(b_kfull, j & 1, err, kErrAttnMma, abort_flag)) break;
-        if (j > 0 && !mbar_wait(b_o, (j - 1) & 1, err, kErrAttnMma, abort_flag)) break;
+      // PV_{j-1}: O += P_{j-1} V_{j-1}
+      auto issue_pv = [&](int jj) -> bool {
+        const int slot = jj & 1;
+        const uint32_t use = (jj >> 1) & 1;
+        if (!mbar_wait(&b_p[slot], use, err, kErrAttnMma, abort_flag)) return false;
+        if (!mbar_wait(&b_vfull[slot], use, err, kErrAttnMma, abort_flag)) return false;
         tc_fence_after();
+        const uint32_t tP = tmem + 64 * slot;
+        const uint32_t vs = v_addr + slot * kKVBytes;
+#pragma unroll
+        for (int k = 0; k < kKTile / 16; ++k)  // keys in steps of 16: P columns advance by 8 words
+          mma_ts(tO, tP + k * 8, sdesc_sw128(vs + k * 16 * 128, kBox, 1024), kIdescO, (jj > 0 || k > 0) ? 1u : 0u);
+        tc_commit(b_o);
+        tc_commit(&b_vempty[slot]);
+        return true;
+      };
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int slot = j & 1;
+        const uint32_t use = (j >> 1) & 1;
+        // S buffer `slot` is free once PV_{j-2} (which read P_{j-2} from it) is complete.
+        if (j >= 2 && !mbar_wait(b_o, (j - 2) & 1, err, kErrAttnMma, abort_flag)) break;
+        if (!mbar_wait(&b_kfull[slot], use, err, kErrAttnMma, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t ks = k_addr + slot * kKVBytes;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // head dim in steps of 16
-          const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
-          mma_ss(tS, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), kIdescS,
+          const uint32_t qoff = (k >> 2) * 2 * kBox + (k & 3) * 32;
+          const uint32_t koff = (k >> 2) * kBox + (k & 3) * 32;
+          mma_ss(tmem + 64 * slot, sdesc_sw128(q_addr + qoff, 16, 1024), sdesc_sw128(ks + koff, 16, 1024), kIdescS,
                  k > 0 ? 1u : 0u);
         }
-        tc_commit(b_s);
-        tc_commit(b_kempty);
-        if (!mbar_wait(b_p, j & 1, err, kErrAttnMma, abort_flag)) break;
-        if (!mbar_wait(b_vfull, j & 1, err, kErrAttnMma, abort_flag)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {  // keys in steps of 16: P columns advance by 8 words
-          mma_ts(tO, tS + k * 8, sdesc_sw128(v_addr + k * 16 * 128, kHalfBytes, 1024), kIdescO,
-                 (j > 0 || k > 0) ? 1u : 0u);
+        tc_commit(&b_s[slot]);
+        tc_commit(&b_kempty[slot]);
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
         }
-        tc_commit(b_o);
-        tc_commit(b_vempty);
       }
+      if (ok) issue_pv(nkv - 1);
       tc_commit(b_drain);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(smem_u32(b_drain), 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
@@ -164,26 +184,45 @@ __global__ void __launch_bounds__(kThreads, 2)
     float l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      ok = mbar_wait(b_s, j & 1, err, kErrAttnSoftmax, abort_flag);
+      const int slot = j & 1;
+      const uint32_t use = (j >> 1) & 1;
+      const uint32_t tS = tmem + 64 * slot + lane_off;
+      ok = mbar_wait(&b_s[slot], use, err, kErrAttnSoftmax, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {  // warp-uniform: TMEM accesses are .sync.aligned
         ok = false;
         break;
       }
       tc_fence_after();
-      const int kvalid = n_tok - j * kTile;  // keys of this step inside the sequence
-      float mx = -INFINITY;
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32f(tS + lane_off + c * 32, v);
+      const int kvalid = n_tok - j * kKTile;  // keys of this step inside the sequence
+      const bool full = kvalid >= kKTile;     // warp-uniform
+      uint32_t sr[64];
+      tmem_ld64(tS, sr);
+      float mxp[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (c * 32 + i < kvalid) mx = fmaxf(mx, v[i]);
+      for (int a = 0; a < 8; ++a) mxp[a] = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) mxp[i & 7] = fmaxf(mxp[i & 7], __uint_as_float(sr[i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i < kvalid) mxp[i & 7] = fmaxf(mxp[i & 7], __uint_as_float(sr[i]));
       }
-      mx *= scale_log2;
+      const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) *
+                       scale_log2;
       const bool grow = mx > m_run + kRescaleThreshold;
       const float m_new = grow ? mx : m_run;
       const float factor = grow ? exp2_approx(m_run - m_new) : 1.0f;  // 0 on the first step
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O may still be accumulating PV_{j-1}: wait for it before rescaling.
+        ok = mbar_wait(b_o, (j - 1) & 1, err, kErrAttnSoftmax, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(tO + lane_off + c * 32, o);
@@ -193,25 +232,32 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       m_run = m_new;
-      float rowsum = 0.f;
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32f(tS + lane_off + c * 32, v);
-        uint32_t pk[16];
+      float sump[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
+      if (full) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int k0 = c * 32 + 2 * i;
-          const float p0 = k0 < kvalid ? exp2_approx(fmaf(v[2 * i], scale_log2, -m_run)) : 0.f;
-          const float p1 = k0 + 1 < kvalid ? exp2_approx(fmaf(v[2 * i + 1], scale_log2, -m_run)) : 0.f;
-          rowsum += p0 + p1;
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = exp2_approx(fmaf(__uint_as_float(sr[2 * i]), scale_log2, -m_run));
+          const float p1 = exp2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), scale_log2, -m_run));
+          sump[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tS + lane_off + c * 16, pk);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = 2 * i < kvalid ? exp2_approx(fmaf(__uint_as_float(sr[2 * i]), scale_log2, -m_run)) : 0.f;
+          const float p1 =
+              2 * i + 1 < kvalid ? exp2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), scale_log2, -m_run)) : 0.f;
+          sump[i & 3] += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
       }
-      l_run = l_run * factor + rowsum;
+      // P_j (BF16 pairs) over the first 32 columns of its S buffer: the A operand of PV_j.
+      tmem_st32(tS, pk);
+      l_run = l_run * factor + ((sump[0] + sump[1]) + (sump[2] + sump[3]));
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(b_p);
+      if (lane == 0) mbar_arrive(&b_p[slot]);
     }
     if (ok) ok = mbar_wait(b_o, (nkv - 1) & 1, err, kErrAttnSoftmax, abort_flag);
     if (__all_sync(0xffffffffu, ok)) {
@@ -219,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float inv_l = 1.0f / l_run;
       const int q = q0 + r;
       bf16* dst = out + (static_cast<int64_t>(b) * n_tok + q) * hidden + h * 128;
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
         float v[32];
         tmem_ld32f(tO + lane_off + c * 32, v);
@@ -245,8 +292,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 }  // namespace
 
-cudaError_t launch_attention(const CUtensorMap& qkv, bf16* o, int batch, int n_tok, int heads, int hidden,
-                             cudaStream_t s, unsigned* err) {
+cudaError_t launch_attention(const bf16* qkv, bf16* o, int batch, int n_tok, int heads, int hidden, cudaStream_t s,
+                             unsigned* err, std::string* emsg) {
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
@@ -254,9 +301,14 @@ cudaError_t launch_attention(const CUtensorMap& qkv, bf16* o, int batch, int n_t
     configured = true;
   }
   if (batch <= 0 || n_tok <= 0) return cudaSuccess;
+  // The tensor map is built here, from the same box constants the kernel's shared-memory
+  // layout and transaction counts use: 64 columns x 64 rows of one branch.
+  CUtensorMap tm;
+  if (!make_tmap_bf16_3d(&tm, qkv, 3 * static_cast<uint64_t>(hidden), n_tok, batch, 64, kBox / 128, emsg))
+    return cudaErrorInvalidValue;
   const float scale_log2 = 1.4426950408889634f / sqrtf(128.0f);
-  dim3 grid((n_tok + kTile - 1) / kTile, heads, batch);
-  attn_kernel<<<grid, kThreads, kSmemBytes, s>>>(qkv, o, n_tok, heads, hidden, scale_log2, err);
+  dim3 grid((n_tok + kQTile - 1) / kQTile, heads, batch);
+  attn_kernel<<<grid, kThreads, kSmemBytes, s>>>(tm, o, n_tok, heads, hidden, scale_log2, err);
   return cudaGetLastError();
 }
 

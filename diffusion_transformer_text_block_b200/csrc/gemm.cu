@@ -9,9 +9,11 @@
 //   warp 1      MMA issuer: one thread issues tcgen05.mma 128xBNx16 (four per 64-wide K
 //               slice) into one of two TMEM accumulators; tcgen05.commit frees the slot
 //               and, after the last K slice, hands the accumulator to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (thread = output row), the fused
-//               element-wise tail of the op, and direct global stores.  Two accumulators
-//               let the epilogue of tile i overlap the main loop of tile i+1.
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (thread = output row; two warps per
+//               TMEM lane quadrant, each owning half of the tile's columns), the fused
+//               element-wise tail of the op, and direct global stores (reductions for the
+//               gated residual).  RoPE angles are read before waiting for the accumulator.  Two accumulators let the epilogue of tile i
+//               overlap the main loop of tile i+1.
 // Tiles are visited in bands of 16 M-tiles (all N-tiles of a band before the next band),
 // so that one band of activations stays in L2 while the weights stream past it.
 //
@@ -29,7 +31,7 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kGroupM = 16;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 
 template <int BN>
 struct GemmShape {
@@ -57,10 +59,15 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const uint32_t (&pk)[16
 }
 
 // ------------------------------------------------------------------------ epilogues
-// tb: TMEM address of this warp's 32 lanes at the accumulator's first column.
+// Eight epilogue warps: warp w reads TMEM lanes 32*(w%4).. (its rows) and owns one half of
+// the tile's columns (`half`).  tb is the TMEM address of the warp's lanes at the
+// accumulator's first column; row is the thread's output row.
 template <int BN>
-__device__ __forceinline__ void epi_f32(const EpiParams& ep, uint32_t tb, int row, int nb) {
-  for (int c = 0; c < BN / 32; ++c) {
+__device__ __forceinline__ void epi_f32(const EpiParams& ep, uint32_t tb, int row, int nb, int half) {
+  constexpr int kChunks = BN / 64;  // 32-column chunks per half
+#pragma unroll
+  for (int cc = 0; cc < kChunks; ++cc) {
+    const int c = half * kChunks + cc;
     const int col = nb * BN + c * 32;
     if (col >= ep.N) break;  // warp-uniform
     float v[32];
@@ -73,83 +80,105 @@ __device__ __forceinline__ void epi_f32(const EpiParams& ep, uint32_t tb, int ro
   }
 }
 
-template <int BN>
-__device__ __forceinline__ void epi_resid(const EpiParams& ep, uint32_t tb, int row, int nb) {
-  for (int c = 0; c < BN / 32; ++c) {
-    const int col = nb * BN + c * 32;
+// x += gate * acc as reductions into the residual stream: every element of x receives
+// exactly one add per launch, so the result is deterministic, and no read of x is waited on.
+__device__ __forceinline__ void red_add_f32x4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void epi_resid(const EpiParams& ep, uint32_t tb, int row, int nb, int half) {
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int c = half * 4 + cc;
+    const int col = nb * 256 + c * 32;
     if (col >= ep.N) break;
     float v[32];
     tmem_ld32f(tb + c * 32, v);
     if (row < ep.M) {
-      float4* x = reinterpret_cast<float4*>(ep.out_f32 + static_cast<int64_t>(row) * ep.N + col);
+      float* x = ep.out_f32 + static_cast<int64_t>(row) * ep.N + col;
       const float4* g = reinterpret_cast<const float4*>(ep.gate + col);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        float4 xv = x[i];
         const float4 gv = __ldg(g + i);
-        xv.x = fmaf(gv.x, v[4 * i + 0], xv.x);
-        xv.y = fmaf(gv.y, v[4 * i + 1], xv.y);
-        xv.z = fmaf(gv.z, v[4 * i + 2], xv.z);
-        xv.w = fmaf(gv.w, v[4 * i + 3], xv.w);
-        x[i] = xv;
+        red_add_f32x4(x + 4 * i, gv.x * v[4 * i], gv.y * v[4 * i + 1], gv.z * v[4 * i + 2], gv.w * v[4 * i + 3]);
       }
     }
   }
 }
 
-// q|k heads: x / sqrt(mean(x^2) + eps) * gain, then rotate pairs (2j, 2j+1) by the token's
-// angle j; v heads are stored unchanged.  Each 128-column head lies in one accumulator
-// half, so the thread owning a row sees the whole head.
-__device__ __forceinline__ void epi_qkv(const EpiParams& ep, uint32_t tb, int row, int nb) {
-  const int tok = row % ep.n_tok;
+// One 128-column head per warp (half = head within the tile).  q|k heads:
+// x / sqrt(mean(x^2) + eps) * gain, then rotate pairs (2j, 2j+1) by the token's angle j;
+// v heads are stored unchanged.
+struct RopePrefetch {
+  float2 cs[32];  // angles of the first 32 rotation pairs (the head's first 64 columns)
+};
+
+__device__ __forceinline__ void qkv_prefetch(const EpiParams& ep, int row, int nb, int half, RopePrefetch& pf) {
+  const int col = nb * 256 + half * 128;
+  if (col < 2 * ep.hidden && col < ep.N) {
+    const float2* rope = ep.rope + static_cast<int64_t>(row % ep.n_tok) * 64;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) pf.cs[i] = __ldg(rope + i);
+  }
+}
+
+__device__ __forceinline__ void epi_qkv(const EpiParams& ep, uint32_t tb, int row, int nb, int half,
+                                        const RopePrefetch& pf) {
   const int ld = 3 * ep.hidden;
-  for (int hh = 0; hh < 2; ++hh) {
-    const int col = nb * 256 + hh * 128;
-    if (col >= ep.N) break;
-    const int region = col / ep.hidden;  // 0 = q, 1 = k, 2 = v
-    const uint32_t th = tb + hh * 128;
-    bf16* dst = ep.out_bf16 + static_cast<int64_t>(row) * ld + col;
-    if (region < 2) {
-      float ss = 0.f;
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32f(th + c * 32, v);
+  const int col = nb * 256 + half * 128;
+  if (col >= ep.N) return;
+  const int region = col / ep.hidden;  // 0 = q, 1 = k, 2 = v
+  const uint32_t th = tb + half * 128;
+  bf16* dst = ep.out_bf16 + static_cast<int64_t>(row) * ld + col;
+  if (region < 2) {
+    float ss[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
-      }
-      const float rinv = rsqrtf(ss * (1.0f / 128.0f) + ep.eps);
-      const float* gain = region == 0 ? ep.q_gain : ep.k_gain;
-      const float2* rope = ep.rope + static_cast<int64_t>(tok) * 64;
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32f(th + c * 32, v);
-        uint32_t pk[16];
+    for (int c = 0; c < 4; ++c) {
+      float v[32];
+      tmem_ld32f(th + c * 32, v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float x0 = v[2 * i] * rinv * __ldg(gain + c * 32 + 2 * i);
-          const float x1 = v[2 * i + 1] * rinv * __ldg(gain + c * 32 + 2 * i + 1);
-          const float2 cs = __ldg(rope + c * 16 + i);
-          pk[i] = pack_bf16x2(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
-        }
-        if (row < ep.M) store_bf16x32(dst + c * 32, pk);
-      }
-    } else {
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32f(th + c * 32, v);
-        uint32_t pk[16];
+      for (int i = 0; i < 32; ++i) ss[i & 3] = fmaf(v[i], v[i], ss[i & 3]);
+    }
+    const float rinv = rsqrtf(((ss[0] + ss[1]) + (ss[2] + ss[3])) * (1.0f / 128.0f) + ep.eps);
+    const float* gain = region == 0 ? ep.q_gain : ep.k_gain;
+    const float2* rope = ep.rope + static_cast<int64_t>(row % ep.n_tok) * 64;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-        if (row < ep.M) store_bf16x32(dst + c * 32, pk);
+    for (int c = 0; c < 4; ++c) {
+      float2 cs[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) cs[i] = c < 2 ? pf.cs[c * 16 + i] : __ldg(rope + c * 16 + i);
+      float v[32];
+      tmem_ld32f(th + c * 32, v);
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float x0 = v[2 * i] * rinv * __ldg(gain + c * 32 + 2 * i);
+        const float x1 = v[2 * i + 1] * rinv * __ldg(gain + c * 32 + 2 * i + 1);
+        pk[i] = pack_bf16x2(x0 * cs[i].x - x1 * cs[i].y, x0 * cs[i].y + x1 * cs[i].x);
       }
+      if (row < ep.M) store_bf16x32(dst + c * 32, pk);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float v[32];
+      tmem_ld32f(th + c * 32, v);
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+      if (row < ep.M) store_bf16x32(dst + c * 32, pk);
     }
   }
 }
 
-// Accumulator columns [0,128) = gate rows f0.., [128,256) = up rows f0.. of the same f.
-__device__ __forceinline__ void epi_swiglu(const EpiParams& ep, uint32_t tb, int row, int nb) {
+// Accumulator columns [0,128) = gate rows f0.., [128,256) = up rows f0.. of the same f;
+// half h handles f0 + 64h .. f0 + 64h + 63.
+__device__ __forceinline__ void epi_swiglu(const EpiParams& ep, uint32_t tb, int row, int nb, int half) {
   const int F = ep.N;
-  for (int c = 0; c < 4; ++c) {
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = half * 2 + cc;
     const int f = nb * 128 + c * 32;
     if (f >= F) break;
     float g[32], u[32];
@@ -166,8 +195,10 @@ __device__ __forceinline__ void epi_swiglu(const EpiParams& ep, uint32_t tb, int
   }
 }
 
-__device__ __forceinline__ void epi_embed(const EpiParams& ep, uint32_t tb, int row, int nb) {
-  for (int c = 0; c < 8; ++c) {
+__device__ __forceinline__ void epi_embed(const EpiParams& ep, uint32_t tb, int row, int nb, int half) {
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int c = half * 4 + cc;
     const int col = nb * 256 + c * 32;
     if (col >= ep.N) break;
     float v[32];
@@ -186,12 +217,15 @@ __device__ __forceinline__ void epi_embed(const EpiParams& ep, uint32_t tb, int 
 }
 
 // Row = b * n_img + token; column j = (dy*2+dx)*32 + ch -> latent [b, 2r+dy, 2c+dx, ch].
-__device__ __forceinline__ void epi_out(const EpiParams& ep, uint32_t tb, int row) {
+// BN = 128: half h handles dy = h.
+__device__ __forceinline__ void epi_out(const EpiParams& ep, uint32_t tb, int row, int half) {
   const int b = row / ep.n_img;
   const int tok = row - b * ep.n_img;
   const int r = tok / ep.grid_w;
   const int cc = tok - r * ep.grid_w;
-  for (int c = 0; c < 4; ++c) {
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int c = half * 2 + q;
     float v[32];
     tmem_ld32f(tb + c * 32, v);
     if (row < ep.M) {
@@ -211,6 +245,7 @@ __device__ __forceinline__ void epi_out(const EpiParams& ep, uint32_t tb, int ro
 }
 
 // ------------------------------------------------------------------------ the kernel
+// Ten warps: three share one SM sub-partition, whose register file caps them at 168 each.
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -242,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], 8);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -348,24 +383,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int quad = warp & 3;          // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;   // which half of the tile's columns it owns
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       int mb, nb;
       tile_coords(tile, num_m, num_n, mb, nb);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      const int row = mb * kBM + quad * 32 + lane;
+      // Operands of the epilogue that do not depend on the accumulator are fetched first.
+      RopePrefetch qp;
+      if constexpr (EPI == kEpiQkv) qkv_prefetch(ep, row, nb, half, qp);
       const bool ok = mbar_wait(&tfull[acc], acc_phase, err, kErrGemmEpilogue, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: TMEM loads are .sync.aligned
       tc_fence_after();
-      const int row = mb * kBM + quad * 32 + lane;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
-      if constexpr (EPI == kEpiF32) epi_f32<BN>(ep, tb, row, nb);
-      if constexpr (EPI == kEpiResid) epi_resid<BN>(ep, tb, row, nb);
-      if constexpr (EPI == kEpiQkv) epi_qkv(ep, tb, row, nb);
-      if constexpr (EPI == kEpiSwiglu) epi_swiglu(ep, tb, row, nb);
-      if constexpr (EPI == kEpiEmbed) epi_embed(ep, tb, row, nb);
-      if constexpr (EPI == kEpiOut) epi_out(ep, tb, row);
+      if constexpr (EPI == kEpiF32) epi_f32<BN>(ep, tb, row, nb, half);
+      if constexpr (EPI == kEpiResid) epi_resid(ep, tb, row, nb, half);
+      if constexpr (EPI == kEpiQkv) epi_qkv(ep, tb, row, nb, half, qp);
+      if constexpr (EPI == kEpiSwiglu) epi_swiglu(ep, tb, row, nb, half);
+      if constexpr (EPI == kEpiEmbed) epi_embed(ep, tb, row, nb, half);
+      if constexpr (EPI == kEpiOut) epi_out(ep, tb, row, half);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);

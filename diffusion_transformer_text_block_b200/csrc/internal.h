@@ -58,9 +58,11 @@ cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& a, const CUtensorMap& b
                         const EpiParams& ep, cudaStream_t s, unsigned* err);
 constexpr int gemm_bn(EpiKind k) { return k == kEpiOut ? 128 : 256; }
 
-// qkv map: 3-D over [batch, n_tok, 3D] BF16 with box {64, 128, 1}.
-cudaError_t launch_attention(const CUtensorMap& qkv, bf16* o, int batch, int n_tok, int heads, int hidden,
-                             cudaStream_t s, unsigned* err);
+// qkv: BF16 [batch, n_tok, 3D] (q | k | v); o: BF16 [batch, n_tok, D].  The launcher builds
+// the kernel's TMA descriptor itself; on a descriptor error it returns cudaErrorInvalidValue
+// with the reason in *emsg.
+cudaError_t launch_attention(const bf16* qkv, bf16* o, int batch, int n_tok, int heads, int hidden, cudaStream_t s,
+                             unsigned* err, std::string* emsg);
 
 // rows of x (FP32, [.., D]) -> h (BF16).  With gather_n_img > 0, output row r reads x row
 // (r / gather_n_img) * gather_n_tok + r % gather_n_img (the image rows of every branch).
