@@ -58,6 +58,24 @@ def step_branch_layers(step, L=42):
     return 2 * L - (len(SKIP) if _slg_on(step % STEPS_PER_IMAGE, STEPS_PER_IMAGE, *SLG) else 0)
 
 
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """The largest `value` over all ranks (the device time of the slowest rank); the input
+    itself when no process group is initialised."""
+    if dist is None or not dist.is_available() or not dist.is_initialized():
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(steps: int, world: int, ms: float, forwards_per_step: int = 2):
+    """Whole-job DiT forwards/s and ms per step: every rank runs `steps` denoising steps of
+    its own image (two forwards each), timed as the max over ranks, `ms` in total."""
+    forwards = forwards_per_step * steps * world
+    return forwards / (ms / 1e3), ms / steps
+
+
 def read_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -284,15 +302,10 @@ def main():
     prof = model.profile_read()
     model.profile_enable(False)
     status = moss.device_status(clear=True)
+    ms = max_over_ranks(ms, dist if world > 1 else None, "cuda")
     if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
-
-    forwards = 2 * args.steps * world
-    value = forwards / (ms / 1e3)
-    ms_per_step = ms / args.steps
+    value, ms_per_step = job_throughput(args.steps, world, ms)
 
     # roofline of the dominant kernel class (largest summed device time)
     N = 4096 + N_TXT
@@ -336,12 +349,8 @@ def main():
             hx.copy_(x, non_blocking=True)
         a1.record(stream)
         torch.cuda.synchronize()
-        ems = a0.elapsed_time(a1)
-        if world > 1:
-            t = torch.tensor([ems], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": 2 * args.e2e_steps * world / (ems / 1e3), "unit": UNIT,
+        ems = max_over_ranks(a0.elapsed_time(a1), dist if world > 1 else None, "cuda")
+        e2e = {"value": job_throughput(args.e2e_steps, world, ems)[0], "unit": UNIT,
                "h2d_bytes_per_step": x.numel() * 4 + tc.numel() * 4 + tu.numel() * 4,
                "d2h_bytes_per_step": x.numel() * 4, "steps": args.e2e_steps}
 

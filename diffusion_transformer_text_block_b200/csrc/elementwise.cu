@@ -200,13 +200,16 @@ __global__ void __launch_bounds__(256) mod_gemv_kernel(const bf16* __restrict__ 
 // ---------------------------------------------------------------------------- RoPE table
 // Angles of the 64 rotation pairs of a 128-wide head: pairs 0..15 (text index), 16..39
 // (patch row), 40..63 (patch column), axis dims 32/48/48, theta 1e4; image token (r, c) at
-// (0, r, c), text token j at (j + 1, 0, 0).  Stored as (cos, sin) in FP32, computed in FP64.
+// (0, r, c), text token j at (j + 1, 0, 0).  Stored as (cos, sin) in FP32, computed in FP64,
+// pair-major: table[j * N + token], so that consecutive tokens (the rows a warp of the QKV
+// epilogue holds) read one contiguous segment.
 __global__ void rope_table_kernel(float2* __restrict__ table, int grid_h, int grid_w, int n_txt) {
   const int n_img = grid_h * grid_w;
+  const int n_tok = n_img + n_txt;
   const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (e >= static_cast<int64_t>(n_img + n_txt) * 64) return;
-  const int tok = static_cast<int>(e / 64);
-  const int j = static_cast<int>(e % 64);
+  if (e >= static_cast<int64_t>(n_tok) * 64) return;
+  const int j = static_cast<int>(e / n_tok);
+  const int tok = static_cast<int>(e % n_tok);
   int p0 = 0, p1 = 0, p2 = 0;
   if (tok < n_img) {
     p1 = tok / grid_w;

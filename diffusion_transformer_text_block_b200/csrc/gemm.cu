@@ -110,16 +110,19 @@ __device__ __forceinline__ void epi_resid(const EpiParams& ep, uint32_t tb, int 
 // One 128-column head per warp (half = head within the tile).  q|k heads:
 // x / sqrt(mean(x^2) + eps) * gain, then rotate pairs (2j, 2j+1) by the token's angle j;
 // v heads are stored unchanged.
+// The RoPE table is pair-major ([64][n_tok]): for a fixed pair the 32 lanes (consecutive
+// tokens) read one contiguous segment.
+constexpr int kRopePrefetch = 16;  // rotation pairs read before the accumulator is ready
 struct RopePrefetch {
-  float2 cs[32];  // angles of the first 32 rotation pairs (the head's first 64 columns)
+  float2 cs[kRopePrefetch];
 };
 
 __device__ __forceinline__ void qkv_prefetch(const EpiParams& ep, int row, int nb, int half, RopePrefetch& pf) {
   const int col = nb * 256 + half * 128;
   if (col < 2 * ep.hidden && col < ep.N) {
-    const float2* rope = ep.rope + static_cast<int64_t>(row % ep.n_tok) * 64;
+    const float2* rope = ep.rope + row % ep.n_tok;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) pf.cs[i] = __ldg(rope + i);
+    for (int i = 0; i < kRopePrefetch; ++i) pf.cs[i] = __ldg(rope + static_cast<int64_t>(i) * ep.n_tok);
   }
 }
 
@@ -142,20 +145,25 @@ __device__ __forceinline__ void epi_qkv(const EpiParams& ep, uint32_t tb, int ro
     }
     const float rinv = rsqrtf(((ss[0] + ss[1]) + (ss[2] + ss[3])) * (1.0f / 128.0f) + ep.eps);
     const float* gain = region == 0 ? ep.q_gain : ep.k_gain;
-    const float2* rope = ep.rope + static_cast<int64_t>(row % ep.n_tok) * 64;
+    const float2* rope = ep.rope + row % ep.n_tok;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       float2 cs[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) cs[i] = c < 2 ? pf.cs[c * 16 + i] : __ldg(rope + c * 16 + i);
+      for (int i = 0; i < 16; ++i)
+        cs[i] = c * 16 + i < kRopePrefetch ? pf.cs[c * 16 + i] : __ldg(rope + static_cast<int64_t>(c * 16 + i) * ep.n_tok);
       float v[32];
       tmem_ld32f(th + c * 32, v);
+      const float4* g4 = reinterpret_cast<const float4*>(gain + c * 32);
       uint32_t pk[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float x0 = v[2 * i] * rinv * __ldg(gain + c * 32 + 2 * i);
-        const float x1 = v[2 * i + 1] * rinv * __ldg(gain + c * 32 + 2 * i + 1);
-        pk[i] = pack_bf16x2(x0 * cs[i].x - x1 * cs[i].y, x0 * cs[i].y + x1 * cs[i].x);
+      for (int i = 0; i < 8; ++i) {
+        const float4 g = __ldg(g4 + i);
+        const float x0 = v[4 * i] * rinv * g.x, x1 = v[4 * i + 1] * rinv * g.y;
+        const float x2 = v[4 * i + 2] * rinv * g.z, x3 = v[4 * i + 3] * rinv * g.w;
+        const float2 ca = cs[2 * i], cb = cs[2 * i + 1];
+        pk[2 * i] = pack_bf16x2(x0 * ca.x - x1 * ca.y, x0 * ca.y + x1 * ca.x);
+        pk[2 * i + 1] = pack_bf16x2(x2 * cb.x - x3 * cb.y, x2 * cb.y + x3 * cb.x);
       }
       if (row < ep.M) store_bf16x32(dst + c * 32, pk);
     }

@@ -30,7 +30,7 @@ struct EpiParams {
   const bf16* bias = nullptr;        // kEpiEmbed, kEpiOut: [N]
   const float* q_gain = nullptr;     // kEpiQkv: [128]
   const float* k_gain = nullptr;     // kEpiQkv: [128]
-  const float2* rope = nullptr;      // kEpiQkv: [n_tok, 64] (cos, sin)
+  const float2* rope = nullptr;      // kEpiQkv: [64, n_tok] (cos, sin), pair-major
   int n_tok = 0;                     // tokens per branch
   int hidden = 0;                    // D
   int n_branch = 0;                  // kEpiEmbed: branches written

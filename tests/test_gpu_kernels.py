@@ -116,3 +116,25 @@ def test_modulation_matches_oracle():
         assert rel_l2(mod, ref) <= 1e-5
     model.close()
     assert_no_device_error()
+
+
+def test_attention_2048_sampled_rows():
+    """The 2048^2 long-sequence shape: 16384 image + 4096 text tokens, batch 2, 24 heads;
+    sampled query rows (tile edges, the image/text boundary, random) against the oracle."""
+    B, N, H = 2, 16384 + 4096, 24
+    D = H * 128
+    g = torch.Generator(device="cuda").manual_seed(11)
+    qkv = torch.randn(B, N, 3 * D, generator=g, device="cuda").to(torch.bfloat16)
+    out = moss.op_attention(qkv, H)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([[0, 63, 64, 127, 128, 16383, 16384, N - 1], rng.integers(0, N, 12)]))
+    got = out[:, rows].float().cpu().numpy()
+    for b in range(B):
+        qb = qkv[b].cpu().double().numpy()
+        q = qb[rows, :D].reshape(len(rows), H, 128).transpose(1, 0, 2)
+        k = qb[:, D:2 * D].reshape(N, H, 128).transpose(1, 0, 2)
+        v = qb[:, 2 * D:].reshape(N, H, 128).transpose(1, 0, 2)
+        ref = o.attention(q, k, v).transpose(1, 0, 2).reshape(len(rows), D)
+        assert rel_l2(got[b], ref) <= 1e-2
+    assert_no_device_error()

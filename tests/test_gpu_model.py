@@ -152,3 +152,19 @@ def test_invalid_requests_launch_nothing():
         model.forward(lat, torch.zeros(2, 17, TINY.hidden, device="cuda"), 64, 64, 0.5)
     assert moss.launch_count() == before
     model.close()
+
+
+def test_block_2048_sampled_rows():
+    """One full-width block at the 2048^2 long-sequence shape (16384 image + 4096 text tokens,
+    batch 2): sampled rows against the oracle's row-restricted block."""
+    gh = gw = 128
+    n_txt = 4096
+    model, x, y, lw, mod, ang = _block_case(WIDE1, 45, gh, gw, n_txt, 2, 0.41)
+    N = gh * gw + n_txt
+    rows = np.array([0, 127, 128, 16383, 16384, N - 1, 9000])
+    for b in range(2):
+        ref = o.block_forward_rows(x[b], lw, mod, ang, rows, WIDE1.heads)
+        assert rel_l2(y[b][rows], ref) <= 1e-2
+        assert rel_l2(y[b][rows] - x[b][rows], ref - x[b][rows]) <= 1e-2
+    model.close()
+    assert_no_device_error()
