@@ -303,8 +303,8 @@ int block_impl(moss_model* m, int l, float* x, int nb, int N, const float* mod_l
   const int M = nb * N;
   std::string e;
   CUtensorMap tm_h, tm_attn, tm_act;
-  if (!make_tmap_bf16_2d(&tm_h, m->h, D, M, 64, 128, &e) || !make_tmap_bf16_2d(&tm_attn, m->attn, D, M, 64, 128, &e) ||
-      !make_tmap_bf16_2d(&tm_act, m->act, F, M, 64, 128, &e))
+  if (!make_tmap_bf16_2d(&tm_h, m->h, D, M, kGemmBoxK, kGemmBoxRows, &e) || !make_tmap_bf16_2d(&tm_attn, m->attn, D, M, kGemmBoxK, kGemmBoxRows, &e) ||
+      !make_tmap_bf16_2d(&tm_act, m->act, F, M, kGemmBoxK, kGemmBoxRows, &e))
     return fail(MOSS_ERR_CUDA, e);
 
   LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(x, mod_l, mod_l + D, m->h, M, D, 0, 0, 1e-6f, s), "ln_modulate 1");
@@ -357,7 +357,7 @@ int forward_impl(moss_model* m, int batch, const float* latent, const float* con
   LAUNCH(m, MOSS_K_OTHER, s, launch_patchify(latent, m->patches, h8, w8, s), "patchify");
   std::string e;
   CUtensorMap tm_p;
-  if (!make_tmap_bf16_2d(&tm_p, m->patches, 128, n_img, 64, 128, &e)) return fail(MOSS_ERR_CUDA, e);
+  if (!make_tmap_bf16_2d(&tm_p, m->patches, 128, n_img, kGemmBoxK, kGemmBoxRows, &e)) return fail(MOSS_ERR_CUDA, e);
   EpiParams pe;
   pe.M = n_img; pe.N = D; pe.K = 128;
   pe.out_f32 = m->x; pe.bias = static_cast<const bf16*>(m->w.img_b);
@@ -389,7 +389,7 @@ int forward_impl(moss_model* m, int batch, const float* latent, const float* con
   const int rows = batch * n_img;
   LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(m->x, fmod, fmod + D, m->h, rows, D, n_img, N, 1e-6f, s), "final ln");
   CUtensorMap tm_hf;
-  if (!make_tmap_bf16_2d(&tm_hf, m->h, D, rows, 64, 128, &e)) return fail(MOSS_ERR_CUDA, e);
+  if (!make_tmap_bf16_2d(&tm_hf, m->h, D, rows, kGemmBoxK, kGemmBoxRows, &e)) return fail(MOSS_ERR_CUDA, e);
   EpiParams oe;
   oe.M = rows; oe.N = 128; oe.K = D;
   oe.out_f32 = v_out; oe.bias = static_cast<const bf16*>(m->w.out_b);
@@ -554,15 +554,15 @@ int moss_model_create(const moss_config* cfg, const moss_weights* w, moss_model*
   const bf16* wd = static_cast<const bf16*>(w->wd);
   for (int l = 0; l < L; ++l) {
     const int64_t dd = static_cast<int64_t>(D) * D, df = static_cast<int64_t>(D) * F;
-    if (!make_tmap_bf16_2d(&m->tm_qkv[l], wqkv + l * 3 * dd, D, 3 * D, 64, 256, &e) ||
-        !make_tmap_bf16_2d(&m->tm_wo[l], wo + l * dd, D, D, 64, 256, &e) ||
-        !make_tmap_bf16_2d(&m->tm_wg[l], wg + l * df, D, F, 64, 128, &e) ||
-        !make_tmap_bf16_2d(&m->tm_wu[l], wu + l * df, D, F, 64, 128, &e) ||
-        !make_tmap_bf16_2d(&m->tm_wd[l], wd + l * df, F, D, 64, 256, &e))
+    if (!make_tmap_bf16_2d(&m->tm_qkv[l], wqkv + l * 3 * dd, D, 3 * D, kGemmBoxK, kGemmBoxRows, &e) ||
+        !make_tmap_bf16_2d(&m->tm_wo[l], wo + l * dd, D, D, kGemmBoxK, kGemmBoxRows, &e) ||
+        !make_tmap_bf16_2d(&m->tm_wg[l], wg + l * df, D, F, kGemmBoxK, kGemmBoxRows, &e) ||
+        !make_tmap_bf16_2d(&m->tm_wu[l], wu + l * df, D, F, kGemmBoxK, kGemmBoxRows, &e) ||
+        !make_tmap_bf16_2d(&m->tm_wd[l], wd + l * df, F, D, kGemmBoxK, kGemmBoxRows, &e))
       return cleanup(MOSS_ERR_CUDA, e);
   }
-  if (!make_tmap_bf16_2d(&m->tm_img, w->img_w, 128, D, 64, 256, &e) ||
-      !make_tmap_bf16_2d(&m->tm_out, w->out_w, D, 128, 64, 128, &e))
+  if (!make_tmap_bf16_2d(&m->tm_img, w->img_w, 128, D, kGemmBoxK, kGemmBoxRows, &e) ||
+      !make_tmap_bf16_2d(&m->tm_out, w->out_w, D, 128, kGemmBoxK, kGemmBoxRows, &e))
     return cleanup(MOSS_ERR_CUDA, e);
   cudaError_t ce = cudaDeviceSynchronize();
   if (ce != cudaSuccess) return cleanup(MOSS_ERR_CUDA, std::string("model creation: ") + cudaGetErrorString(ce));
@@ -772,7 +772,7 @@ int moss_op_gemm_bf16(const void* a, const void* b, float* c, int M, int N, int 
   if (!err) return fail(MOSS_ERR_CUDA, "device error word");
   std::string e;
   CUtensorMap ta, tb;
-  if (!make_tmap_bf16_2d(&ta, a, K, M, 64, 128, &e) || !make_tmap_bf16_2d(&tb, b, K, N, 64, 256, &e))
+  if (!make_tmap_bf16_2d(&ta, a, K, M, kGemmBoxK, kGemmBoxRows, &e) || !make_tmap_bf16_2d(&tb, b, K, N, kGemmBoxK, kGemmBoxRows, &e))
     return fail(MOSS_ERR_CUDA, e);
   EpiParams ep;
   ep.M = M; ep.N = N; ep.K = K; ep.out_f32 = c;

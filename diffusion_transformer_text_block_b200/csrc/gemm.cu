@@ -3,19 +3,26 @@
 //   D[m, n] = sum_k A[m, k] * B[n, k]      A: activations [M, K], B: weights [N, K] (both
 //                                          K-contiguous, BF16), FP32 accumulation in TMEM.
 //
-// Design (one persistent CTA per SM, 192 threads, warp-specialised):
-//   warp 0      TMA producer: 128x64 A tiles and BNx64 B tiles (128-byte swizzle) into a
-//               ring of STAGES shared-memory slots, each guarded by a full/empty mbarrier.
-//   warp 1      MMA issuer: one thread issues tcgen05.mma 128xBNx16 (four per 64-wide K
-//               slice) into one of two TMEM accumulators; tcgen05.commit frees the slot
-//               and, after the last K slice, hands the accumulator to the epilogue.
-//   warps 2..9  epilogue: tcgen05.ld of the accumulator (thread = output row; two warps per
-//               TMEM lane quadrant, each owning half of the tile's columns), the fused
-//               element-wise tail of the op, and direct global stores (reductions for the
-//               gated residual).  RoPE angles are read before waiting for the accumulator.  Two accumulators let the epilogue of tile i
-//               overlap the main loop of tile i+1.
-// Tiles are visited in bands of 16 M-tiles (all N-tiles of a band before the next band),
-// so that one band of activations stays in L2 while the weights stream past it.
+// Main kernel (`gemm_pair_kernel`): persistent CTA pairs (clusters of two CTAs on
+// neighbouring SMs), 320 threads per CTA, one 256 x 256 output tile per pair at a time.
+//   warp 0      TMA producer, in both CTAs: this CTA's 128 rows of A and its 128 rows of the
+//               256-row B tile (128-byte swizzle) into a 6-slot ring; every load is counted on
+//               the even CTA's "full" barrier of the slot.
+//   warp 1      MMA issuer, even CTA only: tcgen05.mma.cta_group::2 256x256x16 (four per 64-wide
+//               K slice) reads A and B halves from both CTAs' shared memory and accumulates the
+//               128 x 256 quarter of each CTA in that CTA's TMEM (two accumulators, 512 columns);
+//               tcgen05.commit frees the slot in both CTAs and hands the accumulator to both
+//               epilogues.
+//   warps 2..9  epilogue, in both CTAs: tcgen05.ld of the accumulator (thread = output row; two
+//               warps per TMEM lane quadrant, each owning half of the tile's columns), the fused
+//               element-wise tail of the op, and direct global stores (reductions for the gated
+//               residual).  The odd CTA's epilogue releases the accumulator on the even CTA's
+//               barrier.  RoPE angles are read before waiting for the accumulator.
+// Each CTA streams half of every B tile, so a pair moves 3/4 of the operand bytes per output
+// of two independent 128-row CTAs, and a 32 KB slot allows a six-deep ring.
+// Tiles are visited in bands of 16 M-tiles (all N-tiles of a band before the next band).
+//
+// The 128 x 128 output projection (`gemm_kernel`, BN = 128) keeps the single-CTA form.
 //
 // Epilogues follow the block of the single-stream DiT (windpaint.ai, MOSS-Image specs:
 // 24 heads of 128, FFN 8192) with the fused tails the sibling DiT names on B200 (SGLang
@@ -35,11 +42,23 @@ constexpr int kThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 
 template <int BN>
 struct GemmShape {
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static_assert(BN == static_cast<int>(kGemmBoxRows), "single-CTA tiles load B with one box");
+  static constexpr int kStages = 6;
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+};
+static_assert(kBM == static_cast<int>(kGemmBoxRows) && kBK == static_cast<int>(kGemmBoxK), "A box");
+
+// CTA-pair tiles: 256 x 256 per pair; per CTA 128 rows of A and 128 rows of B per slot.
+struct PairShape {
+  static constexpr int kStages = 6;
+  static constexpr int kABytes = kBM * kBK * 2;                    // 16 KB
+  static constexpr int kBBytes = static_cast<int>(kGemmBoxRows) * kBK * 2;  // 16 KB, half of B
+  static constexpr int kStageBytes = kABytes + kBBytes;            // 32 KB per CTA
+  static constexpr int kTmemCols = 512;                            // two 256-column accumulators
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 };
 
@@ -274,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_m = (ep.M + kBM - 1) / kBM;
-  const int num_n = EPI == kEpiSwiglu ? (ep.N + 127) / 128 : (ep.N + BN - 1) / BN;
+  const int num_n = (ep.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = ep.K / kBK;
 
@@ -294,7 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (EPI == kEpiSwiglu) tma_prefetch_desc(&tmB2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, S::kTmemCols);
@@ -324,12 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           armed[stage] = static_cast<int>(phase);
           mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
           tma_load_2d(sA + stage * S::kABytes, &tmA, &full[stage], kb * kBK, mb * kBM);
-          if (EPI == kEpiSwiglu) {
-            tma_load_2d(sB + stage * S::kBBytes, &tmB, &full[stage], kb * kBK, nb * 128);
-            tma_load_2d(sB + stage * S::kBBytes + 128 * 128, &tmB2, &full[stage], kb * kBK, nb * 128);
-          } else {
-            tma_load_2d(sB + stage * S::kBBytes, &tmB, &full[stage], kb * kBK, nb * BN);
-          }
+          tma_load_2d(sB + stage * S::kBBytes, &tmB, &full[stage], kb * kBK, nb * BN);
           if (++stage == S::kStages) {
             stage = 0;
             phase ^= 1;
@@ -427,9 +440,196 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------ CTA-pair kernel
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmB2, const EpiParams ep, unsigned* err) {
+  using S = PairShape;
+  constexpr int kTileM = 2 * kBM;  // rows per pair tile
+  constexpr int kTileN = 256;      // accumulator columns per tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S::kStages * S::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kStages * S::kStageBytes);
+  uint64_t* empty = full + S::kStages;
+  uint64_t* tfull = empty + S::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs, 1: its peer
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+  const int num_m = (ep.M + kTileM - 1) / kTileM;
+  const int num_n = EPI == kEpiSwiglu ? (ep.N + 127) / 128 : (ep.N + kTileN - 1) / kTileN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = ep.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 16);  // eight epilogue warps of each CTA (used in the even CTA)
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (EPI == kEpiSwiglu) tma_prefetch_desc(&tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, S::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised and their TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int armed[S::kStages];  // leader: parity of the last phase armed on full[s], -1 = never
+#pragma unroll
+      for (int s2 = 0; s2 < S::kStages; ++s2) armed[s2] = -1;
+      const CUtensorMap* bmap = (EPI == kEpiSwiglu && !leader) ? &tmB2 : &tmB;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, mb, nb);
+        // Even CTA: gate rows (SwiGLU) or B rows 0..127 of the tile; odd CTA: up rows or 128..255.
+        const int brow = EPI == kEpiSwiglu ? nb * 128 : nb * kTileN + static_cast<int>(rank) * 128;
+        const int arow = mb * kTileM + static_cast<int>(rank) * kBM;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, err, kErrGemmProducer, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_leader = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) {
+            armed[stage] = static_cast<int>(phase);
+            mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
+          }
+          tma_load_2d_pair(sA + stage * S::kABytes, &tmA, full_leader, kb * kBK, arow);
+          tma_load_2d_pair(sB + stage * S::kBBytes, bmap, full_leader, kb * kBK, brow);
+          if (++stage == S::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && leader) {
+        // Let the loads already issued land before the CTA can exit (bounded as well).
+        for (int s2 = 0; s2 < S::kStages; ++s2) {
+          if (armed[s2] < 0) continue;
+          const uint32_t a = smem_u32(&full[s2]);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(a, static_cast<uint32_t>(armed[s2])) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      constexpr uint32_t kIdesc = idesc_bf16(kTileM, kTileN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, err, kErrGemmMma, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kTileN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, err, kErrGemmMma, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * S::kABytes);
+          const uint32_t b0 = smem_u32(sB + stage * S::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = sdesc_sw128(a0 + k * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + k * 32, 16, 1024);
+            mma_ss_pair(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair_both(&empty[stage], 0x3);  // the slot in both CTAs
+          if (++stage == S::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) tc_commit_pair_both(&tfull[acc], 0x3);  // both CTAs' epilogues
+      }
+      // Every MMA issued by this thread has completed once `drain` flips: only then may
+      // either CTA release its TMEM, on the normal path and after an abort alike.
+      tc_commit_pair(drain);
+      const uint32_t a = smem_u32(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+    }
+  } else {
+    const int quad = warp & 3;          // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;   // which half of the tile's columns it owns
+    int it = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, mb, nb);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      const int row = mb * kTileM + static_cast<int>(rank) * kBM + quad * 32 + lane;
+      RopePrefetch qp;
+      if constexpr (EPI == kEpiQkv) qkv_prefetch(ep, row, nb, half, qp);
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, err, kErrGemmEpilogue, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: TMEM loads are .sync.aligned
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * kTileN;
+      if constexpr (EPI == kEpiF32) epi_f32<kTileN>(ep, tb, row, nb, half);
+      if constexpr (EPI == kEpiResid) epi_resid(ep, tb, row, nb, half);
+      if constexpr (EPI == kEpiQkv) epi_qkv(ep, tb, row, nb, half, qp);
+      if constexpr (EPI == kEpiSwiglu) epi_swiglu(ep, tb, row, nb, half);
+      if constexpr (EPI == kEpiEmbed) epi_embed(ep, tb, row, nb, half);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&tempty[acc]);
+        else
+          mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the even CTA's MMAs into both TMEMs are complete (drained above)
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, S::kTmemCols);
+  }
+}
+
 template <int BN, int EPI>
-cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const EpiParams& ep,
-                     cudaStream_t s, unsigned* err) {
+cudaError_t launch_single(const CUtensorMap& a, const CUtensorMap& b, const EpiParams& ep, cudaStream_t s,
+                          unsigned* err) {
   using S = GemmShape<BN>;
   static bool configured = false;
   if (!configured) {
@@ -438,12 +638,30 @@ cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorM
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int num_m = (ep.M + kBM - 1) / kBM;
-  const int num_n = EPI == kEpiSwiglu ? (ep.N + 127) / 128 : (ep.N + BN - 1) / BN;
-  const int tiles = num_m * num_n;
+  const int tiles = ((ep.M + kBM - 1) / kBM) * ((ep.N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (grid <= 0) return cudaSuccess;
-  gemm_kernel<BN, EPI><<<grid, kThreads, S::kSmemBytes, s>>>(a, b, b2, ep, err);
+  gemm_kernel<BN, EPI><<<grid, kThreads, S::kSmemBytes, s>>>(a, b, b, ep, err);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const EpiParams& ep,
+                        cudaStream_t s, unsigned* err) {
+  using S = PairShape;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         S::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int num_m = (ep.M + 2 * kBM - 1) / (2 * kBM);
+  const int num_n = EPI == kEpiSwiglu ? (ep.N + 127) / 128 : (ep.N + 255) / 256;
+  const int tiles = num_m * num_n;
+  const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  if (pairs <= 0) return cudaSuccess;
+  gemm_pair_kernel<EPI><<<2 * pairs, kThreads, S::kSmemBytes, s>>>(a, b, b2, ep, err);
   return cudaGetLastError();
 }
 
@@ -452,12 +670,12 @@ cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorM
 cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
                         const EpiParams& ep, cudaStream_t s, unsigned* err) {
   switch (kind) {
-    case kEpiF32: return launch_t<256, kEpiF32>(a, b, b2, ep, s, err);
-    case kEpiQkv: return launch_t<256, kEpiQkv>(a, b, b2, ep, s, err);
-    case kEpiResid: return launch_t<256, kEpiResid>(a, b, b2, ep, s, err);
-    case kEpiSwiglu: return launch_t<256, kEpiSwiglu>(a, b, b2, ep, s, err);
-    case kEpiEmbed: return launch_t<256, kEpiEmbed>(a, b, b2, ep, s, err);
-    case kEpiOut: return launch_t<128, kEpiOut>(a, b, b2, ep, s, err);
+    case kEpiF32: return launch_pair<kEpiF32>(a, b, b2, ep, s, err);
+    case kEpiQkv: return launch_pair<kEpiQkv>(a, b, b2, ep, s, err);
+    case kEpiResid: return launch_pair<kEpiResid>(a, b, b2, ep, s, err);
+    case kEpiSwiglu: return launch_pair<kEpiSwiglu>(a, b, b2, ep, s, err);
+    case kEpiEmbed: return launch_pair<kEpiEmbed>(a, b, b2, ep, s, err);
+    case kEpiOut: return launch_single<128, kEpiOut>(a, b, ep, s, err);
   }
   return cudaErrorInvalidValue;
 }

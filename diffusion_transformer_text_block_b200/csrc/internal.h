@@ -52,11 +52,13 @@ int set_error(int code, const std::string& msg);
 void count_launches(int n);
 
 // ------------------------------------------------------------------ kernels
-// BN = 256 for every epilogue but kEpiOut (BN = 128).  For kEpiSwiglu the B operand is two
-// maps (gate rows, up rows) of box {64, 128}; otherwise box {64, BN}.  A has box {64, 128}.
+// Every GEMM tensor map (A = activations [M, K], B = weights [N, K], BF16) has the box
+// {kGemmBoxK, kGemmBoxRows}: the kernels' shared-memory layout and transaction counts are
+// derived from these two constants.  For kEpiSwiglu, b = gate rows and b2 = up rows.
+constexpr uint32_t kGemmBoxK = 64;
+constexpr uint32_t kGemmBoxRows = 128;
 cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
                         const EpiParams& ep, cudaStream_t s, unsigned* err);
-constexpr int gemm_bn(EpiKind k) { return k == kEpiOut ? 128 : 256; }
 
 // qkv: BF16 [batch, n_tok, 3D] (q | k | v); o: BF16 [batch, n_tok, D].  The launcher builds
 // the kernel's TMA descriptor itself; on a descriptor error it returns cudaErrorInvalidValue
