@@ -76,6 +76,22 @@ def job_throughput(steps: int, world: int, ms: float, forwards_per_step: int = 2
     return forwards / (ms / 1e3), ms / steps
 
 
+def kernel_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu record, or None when the record
+    is missing or the kernel's sources have changed since the counters were taken."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "kernel_traffic.json")))[kernel]
+        h = hashlib.sha256()
+        for f in rec["sources"]:
+            h.update(open(os.path.join(ROOT, f), "rb").read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        return int(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def read_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -325,7 +341,7 @@ def main():
     achieved = fl[dom] * bl / (ms_dom / 1e3) / 1e12
     roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops_sustained"], 4), "traffic": None,
+                "frac": round(achieved / peaks["bf16_tflops_sustained"], 4), "traffic": kernel_traffic(dom),
                 "peak_source": f"{peaks['source']} bf16 sustained",
                 "flop_per_launch": fl[dom] * bl / max(n_dom, 1)}
     step_flops = sum(fl.values()) * bl / args.steps
