@@ -240,9 +240,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive on an mbarrier of another CTA of the cluster (release at cluster scope).
+// Arrive on an mbarrier of another CTA of the cluster.  Default semantics (release at CTA
+// scope): the arrive does not wait for this thread's global stores to become visible to the
+// other CTA, which no consumer of these barriers needs (they order TMEM reads, which
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync already complete).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // TMA tile load whose completion is counted on an mbarrier of either CTA of the pair.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int x, int y) {

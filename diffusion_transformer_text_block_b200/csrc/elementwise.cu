@@ -18,37 +18,60 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ---------------------------------------------------------------------------- LN-modulate
 // h = LN(x) * (1 + scale) + shift: affine-free LayerNorm with biased variance (SGLang
-// cookbook, Qwen-Image 2.1: Lossless LayerNorm modulation).  One warp per row; the row
-// stays in registers (VPL float4 per lane) so mean and variance are exact two-pass sums.
-template <int VPL>
+// cookbook, Qwen-Image 2.1: Lossless LayerNorm modulation).  WPR warps per row; the row stays
+// in registers (VPL float4 per lane) so mean and variance are exact two-pass sums; the
+// warps of a row combine their partial sums through shared memory.  256 threads per block.
+template <int VPL, int WPR>
 __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x, const float* __restrict__ shift,
                                                      const float* __restrict__ scale, bf16* __restrict__ h, int rows,
                                                      int gather_n_img, int gather_n_tok, float eps) {
-  constexpr int D = VPL * 128;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  constexpr int D = VPL * 128 * WPR;
+  constexpr int kRowsPerBlock = 8 / WPR;
+  __shared__ float part[2][8];
+  const int wib = threadIdx.x >> 5;          // warp in block
   const int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
-  int64_t src = warp;
-  if (gather_n_img > 0) src = static_cast<int64_t>(warp / gather_n_img) * gather_n_tok + warp % gather_n_img;
-  const float4* xr = reinterpret_cast<const float4*>(x + src * D);
+  const int rib = wib / WPR;                 // row in block
+  const int sub = wib % WPR;                 // this warp's slice of the row
+  const int row = blockIdx.x * kRowsPerBlock + rib;
+  const bool live = row < rows;              // block-uniform barriers below: no early return
+  int64_t src = row;
+  if (gather_n_img > 0) src = static_cast<int64_t>(row / gather_n_img) * gather_n_tok + row % gather_n_img;
+  const float4* xr = reinterpret_cast<const float4*>(x + src * D) + sub * VPL * 32;
   float4 v[VPL];
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
-    v[i] = __ldcs(xr + lane + 32 * i);
+    v[i] = live ? __ldcs(xr + lane + 32 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
     s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
   }
-  const float mean = warp_sum(s) * (1.0f / D);
+  s = warp_sum(s);
+  if (WPR > 1) {
+    if (lane == 0) part[0][wib] = s;
+    __syncthreads();
+    s = 0.f;
+#pragma unroll
+    for (int k = 0; k < WPR; ++k) s += part[0][rib * WPR + k];
+  }
+  const float mean = s * (1.0f / D);
   float q = 0.f;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
     q += (a * a + b * b) + (c * c + d * d);
   }
-  const float rstd = rsqrtf(warp_sum(q) * (1.0f / D) + eps);
-  uint2* hr = reinterpret_cast<uint2*>(h + static_cast<int64_t>(warp) * D);
-  const float4* sh = reinterpret_cast<const float4*>(shift);
-  const float4* sc = reinterpret_cast<const float4*>(scale);
+  q = warp_sum(q);
+  if (WPR > 1) {
+    if (lane == 0) part[1][wib] = q;
+    __syncthreads();
+    q = 0.f;
+#pragma unroll
+    for (int k = 0; k < WPR; ++k) q += part[1][rib * WPR + k];
+  }
+  if (!live) return;
+  const float rstd = rsqrtf(q * (1.0f / D) + eps);
+  uint2* hr = reinterpret_cast<uint2*>(h + static_cast<int64_t>(row) * D) + sub * VPL * 32;
+  const float4* sh = reinterpret_cast<const float4*>(shift) + sub * VPL * 32;
+  const float4* sc = reinterpret_cast<const float4*>(scale) + sub * VPL * 32;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int j = lane + 32 * i;
@@ -248,11 +271,12 @@ __global__ void patchify_kernel(const float* __restrict__ lat, bf16* __restrict_
   reinterpret_cast<uint2*>(tok)[e] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
 }
 
-template <int VPL>
+template <int VPL, int WPR>
 cudaError_t ln_launch(const float* x, const float* shift, const float* scale, bf16* h, int rows, int gni, int gnt,
                       float eps, cudaStream_t s) {
-  const int blocks = (rows + 7) / 8;
-  ln_mod_kernel<VPL><<<blocks, 256, 0, s>>>(x, shift, scale, h, rows, gni, gnt, eps);
+  constexpr int kRowsPerBlock = 8 / WPR;
+  const int blocks = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
+  ln_mod_kernel<VPL, WPR><<<blocks, 256, 0, s>>>(x, shift, scale, h, rows, gni, gnt, eps);
   return cudaGetLastError();
 }
 
@@ -261,16 +285,17 @@ cudaError_t ln_launch(const float* x, const float* shift, const float* scale, bf
 cudaError_t launch_ln_mod(const float* x, const float* shift, const float* scale, bf16* h, int rows, int dim,
                           int gather_n_img, int gather_n_tok, float eps, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
+  // Rows wider than 2048 are split over two warps (at most 48 values per lane).
   switch (dim / 128) {
-    case 1: return ln_launch<1>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
-    case 2: return ln_launch<2>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
-    case 4: return ln_launch<4>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
-    case 8: return ln_launch<8>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
-    case 16: return ln_launch<16>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
-    case 24: return ln_launch<24>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
-    case 32: return ln_launch<32>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
-    case 48: return ln_launch<48>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
-    case 64: return ln_launch<64>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
+    case 1: return ln_launch<1, 1>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
+    case 2: return ln_launch<2, 1>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
+    case 4: return ln_launch<4, 1>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
+    case 8: return ln_launch<8, 1>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
+    case 16: return ln_launch<8, 2>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
+    case 24: return ln_launch<12, 2>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
+    case 32: return ln_launch<8, 4>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
+    case 48: return ln_launch<12, 4>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
+    case 64: return ln_launch<8, 8>(x, shift, scale, h, rows, gather_n_img, gather_n_tok, eps, s);
     default: return cudaErrorInvalidValue;
   }
 }
