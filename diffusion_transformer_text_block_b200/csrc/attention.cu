@@ -13,7 +13,8 @@
 //   warp 1      one thread issues, in this order, S_0, S_1, PV_0, S_2, PV_1, ...:
 //               S_j = Q K_j^T into S buffer j%2 (operands in shared memory) and
 //               O += P_j V_j (P_j from TMEM, V_j from shared memory as an MN-major operand).
-//               S_j+1 is computed while the softmax warps work on S_j.
+//               S_j+1 is computed while the softmax warps work on S_j.  S_j+2 is issued
+//               right after PV_j without waiting for it: MMAs from one thread run in order.
 //   warps 2..5  softmax, one query row per thread: online softmax in the log2 domain, P_j as
 //               BF16 over the first 32 columns of its S buffer, lazy rescale of O (only when
 //               the running maximum grows by more than 2^8, after waiting for the PV product
@@ -151,8 +152,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int j = 0; j < nkv && ok; ++j) {
         const int slot = j & 1;
         const uint32_t use = (j >> 1) & 1;
-        // S buffer `slot` is free once PV_{j-2} (which read P_{j-2} from it) is complete.
-        if (j >= 2 && !mbar_wait(b_o, (j - 2) & 1, err, kErrAttnMma, abort_flag)) break;
+        // S_j reuses the S buffer whose P_{j-2} the PV_{j-2} product reads.  That product
+        // was issued earlier by this thread, and tcgen05.mma operations issued by one thread
+        // execute in issue order, so it has read P_{j-2} before S_j is written: no wait.
         if (!mbar_wait(&b_kfull[slot], use, err, kErrAttnMma, abort_flag)) break;
         tc_fence_after();
         const uint32_t ks = k_addr + slot * kKVBytes;
