@@ -328,6 +328,14 @@ def main():
     fl = flops_per_branch_layer(N)
     bl = sum(step_branch_layers(i) for i in range(args.steps))
     peaks = read_peaks()
+    # HBM-bound classes: algorithmic bytes over the timed steps.  LN-modulate reads an FP32 row
+    # and writes a BF16 row (2 calls per branch-layer, N rows each, plus the final layer's image
+    # rows per branch); CFG + Euler reads x, v_c, v_u and writes x (16 B per latent element).
+    D = 3072
+    hbm_bytes = {
+        "ln_mod": (2 * bl * N + 2 * 4096 * args.steps) * D * 6.0,
+        "cfg_euler": 16.0 * (HEIGHT // 8) * (WIDTH // 8) * 32 * args.steps,
+    }
     kernels = {}
     for name, (n, tms) in prof.items():
         entry = {"launches": n, "ms": round(tms, 3), "share": round(tms / ms, 4) if ms else None}
@@ -335,6 +343,10 @@ def main():
             tf = fl[name] * bl / (tms / 1e3) / 1e12
             entry["tflops"] = round(tf, 1)
             entry["frac"] = round(tf / peaks["bf16_tflops_sustained"], 4)
+        if name in hbm_bytes and tms > 0:
+            gbs = hbm_bytes[name] / (tms / 1e3) / 1e9
+            entry["gbs"] = round(gbs, 1)
+            entry["hbm_frac"] = round(gbs / peaks["hbm_gbs"], 4)
         kernels[name] = entry
     dom = max((k for k in fl if prof[k][1] > 0), key=lambda k: prof[k][1])
     n_dom, ms_dom = prof[dom]

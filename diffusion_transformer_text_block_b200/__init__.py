@@ -19,8 +19,8 @@ HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "moss_dit.h")
 
 ABI_VERSION = 1
 STATUS = {0: "OK", 1: "INVALID_ARGUMENT", 2: "CUDA", 3: "OOM", 4: "TIMEOUT", 5: "ABI_MISMATCH", 6: "UNSUPPORTED"}
-K_GEMM_QKV, K_GEMM_OPROJ, K_GEMM_GATEUP, K_GEMM_DOWN, K_ATTENTION, K_LN_MOD, K_OTHER = range(7)
-KERNEL_CLASSES = ["gemm_qkv", "gemm_oproj", "gemm_gateup", "gemm_down", "attention", "ln_mod", "other"]
+K_GEMM_QKV, K_GEMM_OPROJ, K_GEMM_GATEUP, K_GEMM_DOWN, K_ATTENTION, K_LN_MOD, K_OTHER, K_CFG_EULER = range(8)
+KERNEL_CLASSES = ["gemm_qkv", "gemm_oproj", "gemm_gateup", "gemm_down", "attention", "ln_mod", "other", "cfg_euler"]
 
 
 class MossError(RuntimeError):

@@ -424,7 +424,7 @@ int step_impl(moss_model* m, float* x, const float* text_c, const float* text_u,
   if (rc) return rc;
   const int64_t n = static_cast<int64_t>(height / 8) * (width / 8) * 32;
   const float* vu = batch == 2 ? m->v + n : m->v;
-  LAUNCH(m, MOSS_K_OTHER, s, launch_cfg_euler(x, m->v, vu, n, batch == 2 ? cfg : 1.0f, sigma, sigma_next, s),
+  LAUNCH(m, MOSS_K_CFG_EULER, s, launch_cfg_euler(x, m->v, vu, n, batch == 2 ? cfg : 1.0f, sigma, sigma_next, s),
          "cfg euler");
   return MOSS_OK;
 }

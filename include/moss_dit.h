@@ -222,7 +222,7 @@ int moss_device_status(int clear);
 /* Kernel classes for profiling. */
 enum {
   MOSS_K_GEMM_QKV = 0, MOSS_K_GEMM_OPROJ = 1, MOSS_K_GEMM_GATEUP = 2, MOSS_K_GEMM_DOWN = 3,
-  MOSS_K_ATTENTION = 4, MOSS_K_LN_MOD = 5, MOSS_K_OTHER = 6, MOSS_K_COUNT = 7
+  MOSS_K_ATTENTION = 4, MOSS_K_LN_MOD = 5, MOSS_K_OTHER = 6, MOSS_K_CFG_EULER = 7, MOSS_K_COUNT = 8
 };
 
 /* Enable (1) or disable (0) CUDA-event timing of every launch of the model's kernels, per

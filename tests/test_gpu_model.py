@@ -168,3 +168,75 @@ def test_block_2048_sampled_rows():
         assert rel_l2(y[b][rows] - x[b][rows], ref - x[b][rows]) <= 1e-2
     model.close()
     assert_no_device_error()
+
+
+@pytest.fixture(scope="module")
+def full_model():
+    """The 42-block, hidden-3072 DiT with ~5B random BF16 weights (drawn on the GPU), sized for
+    the 1024^2 workload: 4096 image + 512 text tokens per branch, batch 2."""
+    from synth import FULL, make_weights
+    w = make_weights(FULL, 2, device="cuda")
+    model = moss.Model(FULL, w, max_tokens=4096 + 512, max_batch=2, max_latent_hw=128 * 128, max_steps=2)
+    yield model, w
+    model.close()
+
+
+def test_full_forward_skip_all_layers_matches_oracle(full_model):
+    """1024^2, all 42 layers skipped: patch embed, final LN-modulate, output projection and
+    unpatchify of the full-size model against the oracle."""
+    from synth import FULL, numpy_weights
+    model, w = full_model
+    lat = make_latent(128, 128, 7, device="cuda")
+    txt = make_text(2, 512, FULL.hidden, 8, device="cuda")
+    skip = list(range(FULL.layers))
+    v = model.forward(lat, txt, 1024, 1024, 0.6, skip_layers=[skip, skip])
+    torch.cuda.synchronize()
+    small = {k: w[k] for k in ("t_w1", "t_b1", "t_w2", "t_b2", "img_w", "img_b", "final_mod_w", "final_mod_b",
+                               "out_w", "out_b")}
+    wn = numpy_weights(small)
+    c = o.conditioning(0.6, wn)
+    img = o.patchify(lat.cpu().double().numpy()) @ wn["img_w"].T + wn["img_b"]
+    ref = o.unpatchify(o.final_layer(img, c, wn), 128, 128)
+    got = v.cpu().double().numpy()
+    for b in range(2):
+        assert rel_l2(got[b], ref) <= 1e-2
+    assert_no_device_error()
+
+
+def test_full_forward_branches_and_determinism(full_model):
+    """1024^2, 42 layers, uncond skipping layer 22: the CFG batch equals each branch run alone
+    (bitwise: every kernel is row-wise or per-branch and free of atomics order effects), and two
+    runs are bitwise identical (run-to-run reproducibility)."""
+    from synth import FULL
+    model, w = full_model
+    lat = make_latent(128, 128, 9, device="cuda")
+    txt = make_text(2, 512, FULL.hidden, 10, device="cuda")
+    v = model.forward(lat, txt, 1024, 1024, 0.77, skip_layers=[[], [22]]).clone()
+    v2 = model.forward(lat, txt, 1024, 1024, 0.77, skip_layers=[[], [22]])
+    assert torch.equal(v, v2)
+    vc = model.forward(lat, txt[:1].contiguous(), 1024, 1024, 0.77, skip_layers=[[]])
+    vu = model.forward(lat, txt[1:].contiguous(), 1024, 1024, 0.77, skip_layers=[[22]])
+    assert torch.equal(v[0], vc[0]) and torch.equal(v[1], vu[0])
+    assert torch.isfinite(v).all()
+    # the skipped layer matters
+    vn = model.forward(lat, txt[1:].contiguous(), 1024, 1024, 0.77, skip_layers=[[]])
+    assert not torch.equal(vn[0], vu[0])
+    assert_no_device_error()
+
+
+def test_full_denoise_step_matches_manual_cfg(full_model):
+    """One 1024^2 denoising step (step 1 of 50: uncond skips layer 22) equals the forward of
+    both branches followed by the CFG + Euler update."""
+    from synth import FULL
+    model, w = full_model
+    x0 = make_latent(128, 128, 11, device="cuda")
+    tc = make_text(1, 512, FULL.hidden, 12, device="cuda")[0].contiguous()
+    tu = make_text(1, 512, FULL.hidden, 13, device="cuda")[0].contiguous()
+    x = x0.clone()
+    model.denoise_step(x, tc, tu, 1024, 1024, 1, 50, 3.0, 5.0, [22], 0.01, 1.0)
+    sig = o.sigma_schedule(50, 5.0)
+    v = model.forward(x0, torch.stack([tc, tu]), 1024, 1024, float(sig[1]), skip_layers=[[], [22]])
+    ref = x0.clone()
+    moss.cfg_euler_step(ref, v[0].contiguous(), v[1].contiguous(), 3.0, float(sig[1]), float(sig[2]))
+    assert torch.equal(x, ref)
+    assert_no_device_error()
