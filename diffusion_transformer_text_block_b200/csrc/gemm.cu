@@ -28,6 +28,8 @@
 // 24 heads of 128, FFN 8192) with the fused tails the sibling DiT names on B200 (SGLang
 // cookbook, Qwen-Image 2.1: Lossless RoPE fusion, Lossless MLP and residual fusion,
 // Lossless Q/K normalization).
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -38,6 +40,7 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kGroupM = 16;
+constexpr int kResidStageBytes = static_cast<int>(kResidBoxCols * kResidBoxRows * 4);  // 2 KB per buffer
 constexpr int kThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 
 template <int BN>
@@ -53,13 +56,19 @@ struct GemmShape {
 static_assert(kBM == static_cast<int>(kGemmBoxRows) && kBK == static_cast<int>(kGemmBoxK), "A box");
 
 // CTA-pair tiles: 256 x 256 per pair; per CTA 128 rows of A and 128 rows of B per slot.
+// Only the gated-residual epilogue stages its reductions in shared memory; the other
+// epilogues leave that space to L1.
+template <int EPI>
 struct PairShape {
   static constexpr int kStages = 6;
   static constexpr int kABytes = kBM * kBK * 2;                    // 16 KB
   static constexpr int kBBytes = static_cast<int>(kGemmBoxRows) * kBK * 2;  // 16 KB, half of B
   static constexpr int kStageBytes = kABytes + kBBytes;            // 32 KB per CTA
   static constexpr int kTmemCols = 512;                            // two 256-column accumulators
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kResidBytes = EPI == kEpiResid ? kEpiWarps * 2 * kResidStageBytes : 0;  // 32 KB
+  static constexpr int kSmemBytes = kStages * kStageBytes + kResidBytes + 1024 + 256;
+  static_assert(kSmemBytes <= 227 * 1024, "pair GEMM shared memory");
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
@@ -99,14 +108,14 @@ __device__ __forceinline__ void epi_f32(const EpiParams& ep, uint32_t tb, int ro
   }
 }
 
-// x += gate * acc as reductions into the residual stream: every element of x receives
-// exactly one add per launch, so the result is deterministic, and no read of x is waited on.
-__device__ __forceinline__ void red_add_f32x4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void epi_resid(const EpiParams& ep, uint32_t tb, int row, int nb, int half) {
+// x += gate * acc through TMA reductions: per 16-column piece of its 32 rows, the warp writes
+// gate * acc to one of its two 2 KB staging buffers (64-byte swizzle: the 16-byte chunk k of
+// row r sits at chunk k ^ ((r >> 1) & 3), conflict-free) and one lane issues an element-wise
+// bulk add into the residual stream.  Each residual element receives exactly one add per
+// launch, so the result is deterministic.
+__device__ __forceinline__ void epi_resid_tma(const EpiParams& ep, const CUtensorMap* xmap, uint32_t tb, int row0,
+                                              int nb, int half, int lane, uint8_t* stage, int& issued) {
+  if (row0 >= ep.M) return;  // the whole warp is past the last row
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
     const int c = half * 4 + cc;
@@ -114,21 +123,38 @@ __device__ __forceinline__ void epi_resid(const EpiParams& ep, uint32_t tb, int 
     if (col >= ep.N) break;
     float v[32];
     tmem_ld32f(tb + c * 32, v);
-    if (row < ep.M) {
-      float* x = ep.out_f32 + static_cast<int64_t>(row) * ep.N + col;
-      const float4* g = reinterpret_cast<const float4*>(ep.gate + col);
+    const float4* g = reinterpret_cast<const float4*>(ep.gate + col);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 gv = __ldg(g + i);
-        red_add_f32x4(x + 4 * i, gv.x * v[4 * i], gv.y * v[4 * i + 1], gv.z * v[4 * i + 2], gv.w * v[4 * i + 3]);
+    for (int i = 0; i < 8; ++i) {
+      const float4 gv = __ldg(g + i);
+      v[4 * i] *= gv.x;
+      v[4 * i + 1] *= gv.y;
+      v[4 * i + 2] *= gv.z;
+      v[4 * i + 3] *= gv.w;
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint8_t* buf = stage + (issued & 1) * kResidStageBytes;
+      if (issued >= 2) {
+        if (lane == 0) bulk_wait_group_read<1>();  // the buffer's previous reduction has read it
+        __syncwarp();
       }
+      float4* rowp = reinterpret_cast<float4*>(buf + lane * 64);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        rowp[k ^ ((lane >> 1) & 3)] =
+            make_float4(v[16 * hh + 4 * k], v[16 * hh + 4 * k + 1], v[16 * hh + 4 * k + 2], v[16 * hh + 4 * k + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_2d(xmap, buf, col + 16 * hh, row0);
+        bulk_commit_group();
+      }
+      ++issued;
     }
   }
 }
 
-// One 128-column head per warp (half = head within the tile).  q|k heads:
-// x / sqrt(mean(x^2) + eps) * gain, then rotate pairs (2j, 2j+1) by the token's angle j;
-// v heads are stored unchanged.
 // The RoPE table is pair-major ([64][n_tok]): for a fixed pair the 32 lanes (consecutive
 // tokens) read one contiguous segment.
 constexpr int kRopePrefetch = 16;  // rotation pairs read before the accumulator is ready
@@ -421,7 +447,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
       if constexpr (EPI == kEpiF32) epi_f32<BN>(ep, tb, row, nb, half);
-      if constexpr (EPI == kEpiResid) epi_resid(ep, tb, row, nb, half);
       if constexpr (EPI == kEpiQkv) epi_qkv(ep, tb, row, nb, half, qp);
       if constexpr (EPI == kEpiSwiglu) epi_swiglu(ep, tb, row, nb, half);
       if constexpr (EPI == kEpiEmbed) epi_embed(ep, tb, row, nb, half);
@@ -444,15 +469,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmB2, const EpiParams ep, unsigned* err) {
-  using S = PairShape;
+                     const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmX,
+                     const EpiParams ep, unsigned* err) {
+  using S = PairShape<EPI>;
   constexpr int kTileM = 2 * kBM;  // rows per pair tile
   constexpr int kTileN = 256;      // accumulator columns per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S::kStages * S::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kStages * S::kStageBytes);
+  uint8_t* sResid = smem + S::kStages * S::kStageBytes;  // 1024-aligned: kStageBytes is 32 KB
+  uint64_t* full = reinterpret_cast<uint64_t*>(sResid + S::kResidBytes);
   uint64_t* empty = full + S::kStages;
   uint64_t* tfull = empty + S::kStages;
   uint64_t* tempty = tfull + 2;
@@ -488,6 +515,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     if (EPI == kEpiSwiglu) tma_prefetch_desc(&tmB2);
+    if (EPI == kEpiResid) tma_prefetch_desc(&tmX);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, S::kTmemCols);
@@ -589,13 +617,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else {
     const int quad = warp & 3;          // TMEM lane quadrant this warp may access
     const int half = (warp - 2) >> 2;   // which half of the tile's columns it owns
+    uint8_t* stage = sResid + (warp - 2) * 2 * kResidStageBytes;
+    int issued = 0;                     // residual reductions this warp has issued
     int it = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
       int mb, nb;
       tile_coords(tile, num_m, num_n, mb, nb);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      const int row = mb * kTileM + static_cast<int>(rank) * kBM + quad * 32 + lane;
+      const int row0 = mb * kTileM + static_cast<int>(rank) * kBM + quad * 32;
+      const int row = row0 + lane;
       RopePrefetch qp;
       if constexpr (EPI == kEpiQkv) qkv_prefetch(ep, row, nb, half, qp);
       const bool ok = mbar_wait(&tfull[acc], acc_phase, err, kErrGemmEpilogue, abort_flag);
@@ -603,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * kTileN;
       if constexpr (EPI == kEpiF32) epi_f32<kTileN>(ep, tb, row, nb, half);
-      if constexpr (EPI == kEpiResid) epi_resid(ep, tb, row, nb, half);
+      if constexpr (EPI == kEpiResid) epi_resid_tma(ep, &tmX, tb, row0, nb, half, lane, stage, issued);
       if constexpr (EPI == kEpiQkv) epi_qkv(ep, tb, row, nb, half, qp);
       if constexpr (EPI == kEpiSwiglu) epi_swiglu(ep, tb, row, nb, half);
       if constexpr (EPI == kEpiEmbed) epi_embed(ep, tb, row, nb, half);
@@ -616,6 +647,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
       }
     }
+    // The reductions must have read their staging buffers (and completed) before exit.
+    if (EPI == kEpiResid && lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -648,7 +682,7 @@ cudaError_t launch_single(const CUtensorMap& a, const CUtensorMap& b, const EpiP
 template <int EPI>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const EpiParams& ep,
                         cudaStream_t s, unsigned* err) {
-  using S = PairShape;
+  using S = PairShape<EPI>;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -656,12 +690,19 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtens
     if (e != cudaSuccess) return e;
     configured = true;
   }
+  // The residual stream's reduction descriptor is built here from the same box constants the
+  // epilogue's staging layout uses.
+  CUtensorMap xmap;
+  std::memset(&xmap, 0, sizeof xmap);
+  if (EPI == kEpiResid &&
+      !make_tmap_f32_2d_sw64(&xmap, ep.out_f32, ep.N, ep.M, kResidBoxCols, kResidBoxRows, nullptr))
+    return cudaErrorInvalidValue;
   const int num_m = (ep.M + 2 * kBM - 1) / (2 * kBM);
   const int num_n = EPI == kEpiSwiglu ? (ep.N + 127) / 128 : (ep.N + 255) / 256;
   const int tiles = num_m * num_n;
   const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
   if (pairs <= 0) return cudaSuccess;
-  gemm_pair_kernel<EPI><<<2 * pairs, kThreads, S::kSmemBytes, s>>>(a, b, b2, ep, err);
+  gemm_pair_kernel<EPI><<<2 * pairs, kThreads, S::kSmemBytes, s>>>(a, b, b2, xmap, ep, err);
   return cudaGetLastError();
 }
 

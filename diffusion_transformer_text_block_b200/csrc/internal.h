@@ -12,6 +12,10 @@ namespace moss {
 
 using bf16 = __nv_bfloat16;
 
+// Residual reduction tiles of the gated-residual epilogue: 16 FP32 columns x 32 rows.
+constexpr uint32_t kResidBoxCols = 16;
+constexpr uint32_t kResidBoxRows = 32;
+
 // ------------------------------------------------------------------ GEMM epilogue kinds
 enum EpiKind : int {
   kEpiF32 = 0,     // C = acc (FP32), test / library GEMM
@@ -43,6 +47,10 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
                        uint32_t box_outer, std::string* err);
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
                        uint32_t box_inner, uint32_t box_mid, std::string* err);
+
+// FP32 [outer, inner] map with a 64-byte swizzle, for TMA reductions into the residual stream.
+bool make_tmap_f32_2d_sw64(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                           uint32_t box_outer, std::string* err);
 
 int num_sms();
 
