@@ -37,6 +37,8 @@ Readings taken where the pages are silent (each repeated where it is used):
   R13 A skipped layer is the identity on that branch's residual stream.
   R14 Initial noise: Philox4x32-10 (Salmon et al., SC'11) keyed by the seed, counter =
       element-group index, Box-Muller on 23-bit uniforms.
+  R15 The two CFG branches each attend over their own prompt tokens; their lengths may
+      differ and are never padded.
 """
 from __future__ import annotations
 
@@ -427,9 +429,12 @@ def sample(w: dict, heads: int, height: int, width: int, text_c: np.ndarray, tex
             x = euler_update(x, v_c.astype(F32), sig[i], sig[i + 1])
             continue
         skip_u = tuple(uncond_skip_layers) if slg_active(i, steps, slg_start, slg_stop) else ()
-        texts = np.stack([text_c, text_u])
-        v = dit_forward(x, texts, t, [(), skip_u], w, heads, head_dim).astype(F32)
-        x = cfg_euler(x, v[0], v[1], cfg, sig[i], sig[i + 1])
+        # Each branch attends over its own prompt: the two may differ in length (the default
+        # negative prompt is empty), with no padding ([SGL-MOSS] 5: samples of different text
+        # length run without padding).
+        v_c = dit_forward(x, np.asarray(text_c)[None], t, [()], w, heads, head_dim)[0].astype(F32)
+        v_u = dit_forward(x, np.asarray(text_u)[None], t, [skip_u], w, heads, head_dim)[0].astype(F32)
+        x = cfg_euler(x, v_c, v_u, cfg, sig[i], sig[i + 1])
     return x
 
 

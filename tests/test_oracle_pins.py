@@ -441,3 +441,26 @@ def test_block_rows_equals_full_block():
     rows = [0, 5, 17, 31]
     np.testing.assert_allclose(o.block_forward_rows(x, lw, mod, ang, rows, TINY.heads), full[rows],
                                rtol=1e-12, atol=1e-12)
+
+
+def test_sampler_branches_with_different_text_lengths():
+    """Each branch uses its own prompt length: the sampler with a short negative prompt equals
+    the guided Euler update of two separate single-branch forwards."""
+    w = numpy_weights(make_weights(TINY, 15))
+    rng = np.random.default_rng(15)
+    tc = rng.standard_normal((16, TINY.hidden))
+    tu = rng.standard_normal((5, TINY.hidden))
+    x0 = rng.standard_normal((8, 8, 32)).astype(np.float32)
+    out = o.sample(w, TINY.heads, 64, 64, tc, tu, steps=2, cfg=3.0, uncond_skip_layers=(1,), x0=x0)
+    sig = o.sigma_schedule(2, 5.0)
+    x = x0
+    for i in range(2):
+        su = (1,) if o.slg_active(i, 2, 0.01, 1.0) else ()
+        vc = o.dit_forward(x, tc[None], float(sig[i]), [()], w, TINY.heads)[0].astype(np.float32)
+        vu = o.dit_forward(x, tu[None], float(sig[i]), [su], w, TINY.heads)[0].astype(np.float32)
+        x = o.cfg_euler(x, vc, vu, 3.0, sig[i], sig[i + 1])
+    np.testing.assert_array_equal(out, x)
+    # padding the short prompt with zero tokens changes the result (no padding semantics)
+    tu_pad = np.concatenate([tu, np.zeros((11, TINY.hidden))])
+    out_pad = o.sample(w, TINY.heads, 64, 64, tc, tu_pad, steps=2, cfg=3.0, uncond_skip_layers=(1,), x0=x0)
+    assert not np.allclose(out, out_pad)
