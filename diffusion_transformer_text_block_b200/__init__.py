@@ -64,8 +64,8 @@ _SIGS = {
     "moss_sigma_schedule": (_I, [_I, _D, ctypes.POINTER(_F)]),
     "moss_slg_active": (_I, [_I, _I, _D, _D]),
     "moss_init_noise": (_I, [_P, _I64, ctypes.c_uint64, _P]),
-    "moss_denoise_step": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _D, _P, _I, _D, _D, _P]),
-    "moss_sample": (_I, [_P, _I, _F, _D, ctypes.c_uint64, _P, _I, _D, _D, _P, _P, _I, _I, _I, _P, _P]),
+    "moss_denoise_step": (_I, [_P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _F, _D, _P, _I, _D, _D, _P]),
+    "moss_sample": (_I, [_P, _I, _F, _D, ctypes.c_uint64, _P, _I, _D, _D, _P, _I, _P, _I, _I, _I, _P, _P]),
     "moss_device_status": (_I, [_I]),
     "moss_profile_enable": (_I, [_P, _I]),
     "moss_profile_read": (_I, [_P, _I, ctypes.POINTER(_I64), ctypes.POINTER(_D)]),
@@ -293,12 +293,13 @@ class Model:
     def denoise_step(self, x, text_c, text_u, height: int, width: int, step: int, steps: int = 50, cfg: float = 3.0,
                      shift: float = 5.0, uncond_skip_layers: Sequence[int] = (22,), slg_start: float = 0.01,
                      slg_stop: float = 1.0, stream=None):
+        """text_c [n_c, D] and text_u [n_u, D] may differ in length; text_u may be None when cfg == 1."""
         import torch
-        n_txt = text_c.shape[0]
         arr, n = _skip_array([list(uncond_skip_layers)])
         f = torch.float32
-        _check(lib().moss_denoise_step(self._h, _ptr(x, f, "x"), _ptr(text_c, f, "text_c"),
-                                       _ptr(text_u, f, "text_u") if text_u is not None else None, n_txt, height,
+        n_u = text_u.shape[0] if text_u is not None else 0
+        _check(lib().moss_denoise_step(self._h, _ptr(x, f, "x"), _ptr(text_c, f, "text_c"), text_c.shape[0],
+                                       _ptr(text_u, f, "text_u") if text_u is not None else None, n_u, height,
                                        width, step, steps, cfg, shift, arr, n, slg_start, slg_stop, _stream(stream)))
         return x
 
@@ -308,12 +309,13 @@ class Model:
         import torch
         if out is None:
             out = torch.empty(height // 8, width // 8, 32, device=text_c.device, dtype=torch.float32)
-        n_txt = text_c.shape[0]
         arr, n = _skip_array([list(uncond_skip_layers)])
         f = torch.float32
+        n_u = text_u.shape[0] if text_u is not None else 0
         _check(lib().moss_sample(self._h, steps, cfg, shift, seed, arr, n, slg_start, slg_stop,
-                                 _ptr(text_c, f, "text_c"), _ptr(text_u, f, "text_u") if text_u is not None else None,
-                                 n_txt, height, width, _ptr(out, f, "out"), _stream(stream)))
+                                 _ptr(text_c, f, "text_c"), text_c.shape[0],
+                                 _ptr(text_u, f, "text_u") if text_u is not None else None, n_u,
+                                 height, width, _ptr(out, f, "out"), _stream(stream)))
         return out
 
     def modulation(self, t: float, stream=None):

@@ -203,6 +203,7 @@ struct moss_model {
   float* tvals = nullptr;
   int64_t mod_stride = 0;
   int rope_gh = -1, rope_gw = -1, rope_nt = -1;
+  int rope_n = 0;  // tokens of the cached RoPE table (its pair-row stride)
   unsigned* err = nullptr;
   // weight descriptors
   std::vector<CUtensorMap> tm_qkv, tm_wo, tm_wg, tm_wu, tm_wd;
@@ -295,6 +296,7 @@ int ensure_rope(moss_model* m, int gh, int gw, int nt, cudaStream_t s) {
   m->rope_gh = gh;
   m->rope_gw = gw;
   m->rope_nt = nt;
+  m->rope_n = gh * gw + nt;
   return MOSS_OK;
 }
 
@@ -319,11 +321,20 @@ int compute_modulation(moss_model* m, const float* ts_host, int T, cudaStream_t 
   return MOSS_OK;
 }
 
-// One joint block over nb branches of x (rows [nb * N, D]); mod_l = [6D] of this layer.
-int block_impl(moss_model* m, int l, float* x, int nb, int N, const float* mod_l, cudaStream_t s) {
+// One joint block over consecutive branches of the packed stream x (branch i has lens[i]
+// rows, [image; text]); mod_l = [6D] of this layer.  Branches of different lengths are
+// supported for two branches (the QKV epilogue maps rows past the first branch onto the
+// second branch's tokens; attention runs per branch).
+int block_impl(moss_model* m, int l, float* x, const std::vector<int>& lens, const float* mod_l, cudaStream_t s) {
   const moss_config& c = m->cfg;
   const int D = c.hidden, F = c.ffn, H = c.heads;
-  const int M = nb * N;
+  const int nb = static_cast<int>(lens.size());
+  bool equal = true;
+  int M = 0;
+  for (int n : lens) {
+    M += n;
+    equal = equal && n == lens[0];
+  }
   std::string e;
   CUtensorMap tm_h, tm_attn, tm_act;
   if (!make_tmap_bf16_2d(&tm_h, m->h, D, M, kGemmBoxK, kGemmBoxRows, &e) || !make_tmap_bf16_2d(&tm_attn, m->attn, D, M, kGemmBoxK, kGemmBoxRows, &e) ||
@@ -337,11 +348,23 @@ int block_impl(moss_model* m, int l, float* x, int nb, int N, const float* mod_l
   q.out_bf16 = m->qkv;
   q.q_gain = m->w.q_gain + static_cast<int64_t>(l) * 128;
   q.k_gain = m->w.k_gain + static_cast<int64_t>(l) * 128;
-  q.rope = m->rope; q.n_tok = N; q.hidden = D;
+  q.rope = m->rope; q.n_tok = lens[0]; q.hidden = D;
+  q.split_rows = equal ? 0 : lens[0];
+  q.rope_stride = m->rope_n;
   LAUNCH(m, MOSS_K_GEMM_QKV, s, launch_gemm(kEpiQkv, tm_h, m->tm_qkv[l], m->tm_qkv[l], q, s, m->err), "qkv gemm");
 
-  LAUNCH(m, MOSS_K_ATTENTION, s, launch_attention(m->qkv, m->attn, nb, N, H, D, s, m->err, &e),
-         e.empty() ? "attention" : e.c_str());
+  if (equal) {
+    LAUNCH(m, MOSS_K_ATTENTION, s, launch_attention(m->qkv, m->attn, nb, lens[0], H, D, s, m->err, &e),
+           e.empty() ? "attention" : e.c_str());
+  } else {
+    int64_t off = 0;
+    for (int i = 0; i < nb; ++i) {
+      LAUNCH(m, MOSS_K_ATTENTION, s,
+             launch_attention(m->qkv + off * 3 * D, m->attn + off * D, 1, lens[i], H, D, s, m->err, &e),
+             e.empty() ? "attention" : e.c_str());
+      off += lens[i];
+    }
+  }
 
   EpiParams o;
   o.M = M; o.N = D; o.K = D;
@@ -366,15 +389,29 @@ int block_impl(moss_model* m, int l, float* x, int nb, int N, const float* mod_l
   return MOSS_OK;
 }
 
-// The DiT for `batch` branches sharing `latent`; skip[b] = sorted layer ids branch b skips.
-int forward_impl(moss_model* m, int batch, const float* latent, const float* const* texts, int n_txt, int height,
-                 int width, const float* mod, const std::vector<std::vector<char>>& skip, float* v_out,
+// The DiT for `batch` branches sharing `latent`, branch b with n_txts[b] text tokens (equal
+// lengths for any batch, or two branches of different lengths); the branches' rows are packed
+// back to back in the residual stream.  skip[b][l] != 0: branch b skips layer l.
+int forward_impl(moss_model* m, int batch, const float* latent, const float* const* texts, const int* n_txts,
+                 int height, int width, const float* mod, const std::vector<std::vector<char>>& skip, float* v_out,
                  cudaStream_t s) {
   const moss_config& c = m->cfg;
   const int D = c.hidden, L = c.layers;
   const int h8 = height / 8, w8 = width / 8, gh = height / 16, gw = width / 16;
-  const int n_img = gh * gw, N = n_img + n_txt;
-  int rc = ensure_rope(m, gh, gw, n_txt, s);
+  const int n_img = gh * gw;
+  std::vector<int> lens(batch);
+  std::vector<int64_t> off(batch + 1, 0);
+  int n_txt_max = 0;
+  bool equal = true;
+  for (int b = 0; b < batch; ++b) {
+    lens[b] = n_img + n_txts[b];
+    off[b + 1] = off[b] + lens[b];
+    n_txt_max = std::max(n_txt_max, n_txts[b]);
+    equal = equal && n_txts[b] == n_txts[0];
+  }
+  if (!equal && batch > 2)
+    return fail(MOSS_ERR_UNSUPPORTED, "branches of different text lengths are supported for two branches");
+  int rc = ensure_rope(m, gh, gw, n_txt_max, s);
   if (rc) return rc;
 
   LAUNCH(m, MOSS_K_OTHER, s, launch_patchify(latent, m->patches, h8, w8, s), "patchify");
@@ -384,12 +421,12 @@ int forward_impl(moss_model* m, int batch, const float* latent, const float* con
   EpiParams pe;
   pe.M = n_img; pe.N = D; pe.K = 128;
   pe.out_f32 = m->x; pe.bias = static_cast<const bf16*>(m->w.img_b);
-  pe.n_tok = N; pe.n_branch = batch;
+  pe.n_tok = lens[0]; pe.n_branch = batch;  // branch b's rows start at b * lens[0] (batch <= 2 if ragged)
   LAUNCH(m, MOSS_K_OTHER, s, launch_gemm(kEpiEmbed, tm_p, m->tm_img, m->tm_img, pe, s, m->err), "patch embed");
   for (int b = 0; b < batch; ++b) {
-    if (n_txt == 0) continue;
-    MOSS_CUDA(cudaMemcpyAsync(m->x + (static_cast<int64_t>(b) * N + n_img) * D, texts[b],
-                              sizeof(float) * static_cast<size_t>(n_txt) * D, cudaMemcpyDeviceToDevice, s),
+    if (n_txts[b] == 0) continue;
+    MOSS_CUDA(cudaMemcpyAsync(m->x + (off[b] + n_img) * D, texts[b], sizeof(float) * static_cast<size_t>(n_txts[b]) * D,
+                              cudaMemcpyDeviceToDevice, s),
               "copy text states");
   }
 
@@ -402,7 +439,8 @@ int forward_impl(moss_model* m, int batch, const float* latent, const float* con
       }
       int e2 = b;
       while (e2 < batch && !skip[e2][l]) ++e2;
-      rc = block_impl(m, l, m->x + static_cast<int64_t>(b) * N * D, e2 - b, N, mod + static_cast<int64_t>(l) * 6 * D, s);
+      const std::vector<int> run(lens.begin() + b, lens.begin() + e2);
+      rc = block_impl(m, l, m->x + off[b] * D, run, mod + static_cast<int64_t>(l) * 6 * D, s);
       if (rc) return rc;
       b = e2;
     }
@@ -410,7 +448,9 @@ int forward_impl(moss_model* m, int batch, const float* latent, const float* con
 
   const float* fmod = mod + static_cast<int64_t>(L) * 6 * D;
   const int rows = batch * n_img;
-  LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(m->x, fmod, fmod + D, m->h, rows, D, n_img, N, 1e-6f, s), "final ln");
+  // Image rows of branch b start at b * lens[0] (equal lengths, or two branches).
+  LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(m->x, fmod, fmod + D, m->h, rows, D, n_img, lens[0], 1e-6f, s),
+         "final ln");
   CUtensorMap tm_hf;
   if (!make_tmap_bf16_2d(&tm_hf, m->h, D, rows, kGemmBoxK, kGemmBoxRows, &e)) return fail(MOSS_ERR_CUDA, e);
   EpiParams oe;
@@ -436,14 +476,15 @@ int parse_skips(moss_model* m, int batch, const int* skip_layers, int n_skip, st
   return MOSS_OK;
 }
 
-int step_impl(moss_model* m, float* x, const float* text_c, const float* text_u, int n_txt, int height, int width,
-              float sigma, float sigma_next, float cfg, const std::vector<char>& uskip, const float* mod,
-              cudaStream_t s) {
+int step_impl(moss_model* m, float* x, const float* text_c, int n_txt_c, const float* text_u, int n_txt_u,
+              int height, int width, float sigma, float sigma_next, float cfg, const std::vector<char>& uskip,
+              const float* mod, cudaStream_t s) {
   const int batch = cfg == 1.0f ? 1 : 2;
   std::vector<std::vector<char>> skips(batch, std::vector<char>(m->cfg.layers, 0));
   if (batch == 2) skips[1] = uskip;
   const float* texts[2] = {text_c, text_u};
-  int rc = forward_impl(m, batch, x, texts, n_txt, height, width, mod, skips, m->v, s);
+  const int n_txts[2] = {n_txt_c, n_txt_u};
+  int rc = forward_impl(m, batch, x, texts, n_txts, height, width, mod, skips, m->v, s);
   if (rc) return rc;
   const int64_t n = static_cast<int64_t>(height / 8) * (width / 8) * 32;
   const float* vu = batch == 2 ? m->v + n : m->v;
@@ -617,7 +658,8 @@ int moss_dit_block_forward(moss_model* m, int layer, float* x, int batch, int gr
   rc = ensure_rope(m, grid_h, grid_w, n_txt, s);
   if (rc) return rc;
   const int D = m->cfg.hidden;
-  return block_impl(m, layer, x, batch, grid_h * grid_w + n_txt, m->mod + static_cast<int64_t>(layer) * 6 * D, s);
+  const std::vector<int> lens(batch, grid_h * grid_w + n_txt);
+  return block_impl(m, layer, x, lens, m->mod + static_cast<int64_t>(layer) * 6 * D, s);
 }
 
 int moss_dit_forward(moss_model* m, int batch, const float* latent, const float* text_states, int n_txt, int height,
@@ -639,7 +681,8 @@ int moss_dit_forward(moss_model* m, int batch, const float* latent, const float*
   if (rc) return rc;
   std::vector<const float*> texts(batch);
   for (int b = 0; b < batch; ++b) texts[b] = text_states + static_cast<int64_t>(b) * n_txt * m->cfg.hidden;
-  return forward_impl(m, batch, latent, texts.data(), n_txt, height, width, m->mod, skips, v_out, s);
+  const std::vector<int> n_txts(batch, n_txt);
+  return forward_impl(m, batch, latent, texts.data(), n_txts.data(), height, width, m->mod, skips, v_out, s);
 }
 
 int moss_cfg_euler_step(float* x, const float* v_c, const float* v_u, int64_t n, float cfg, float sigma,
@@ -679,15 +722,18 @@ int moss_init_noise(float* x, int64_t n, uint64_t seed, void* stream) {
   return e == cudaSuccess ? MOSS_OK : cuda_fail(e, "noise");
 }
 
-static int check_step_args(moss_model* m, float* x, const float* text_c, const float* text_u, int n_txt, int height,
-                           int width, float cfg, const int* uskip, int n_skip, std::vector<char>* skipv) {
-  if (!m || !x || (n_txt > 0 && !text_c) || (cfg != 1.0f && n_txt > 0 && !text_u))
+static int check_step_args(moss_model* m, float* x, const float* text_c, int n_txt_c, const float* text_u,
+                           int n_txt_u, int height, int width, float cfg, const int* uskip, int n_skip,
+                           std::vector<char>* skipv) {
+  if (!m || !x || (n_txt_c > 0 && !text_c) || (cfg != 1.0f && n_txt_u > 0 && !text_u))
     return fail(MOSS_ERR_INVALID_ARGUMENT, "model, x and text states must not be NULL");
+  if (n_txt_c < 0 || n_txt_u < 0) return fail(MOSS_ERR_INVALID_ARGUMENT, "text lengths must be >= 0");
   if (!aligned16(x) || (text_c && !aligned16(text_c)) || (text_u && !aligned16(text_u)))
     return fail(MOSS_ERR_INVALID_ARGUMENT, "device buffers must be 16-byte aligned");
   int rc = check_size(height, width);
   if (rc) return rc;
-  rc = check_tokens(m, cfg == 1.0f ? 1 : 2, height / 16, width / 16, n_txt);
+  rc = check_tokens(m, cfg == 1.0f ? 1 : 2, height / 16, width / 16,
+                    cfg == 1.0f ? n_txt_c : std::max(n_txt_c, n_txt_u));
   if (rc) return rc;
   std::vector<std::vector<char>> sk;
   rc = parse_skips(m, 1, uskip, n_skip, &sk);
@@ -696,14 +742,15 @@ static int check_step_args(moss_model* m, float* x, const float* text_c, const f
   return MOSS_OK;
 }
 
-int moss_denoise_step(moss_model* m, float* x, const float* text_c, const float* text_u, int n_txt, int height,
-                      int width, int step, int steps, float cfg, double shift, const int* uncond_skip_layers,
-                      int n_skip, double slg_start, double slg_stop, void* stream) {
+int moss_denoise_step(moss_model* m, float* x, const float* text_c, int n_txt_c, const float* text_u, int n_txt_u,
+                      int height, int width, int step, int steps, float cfg, double shift,
+                      const int* uncond_skip_layers, int n_skip, double slg_start, double slg_stop, void* stream) {
   g_last_error.clear();
   if (steps < 1 || step < 0 || step >= steps || !(shift > 0.0))
     return fail(MOSS_ERR_INVALID_ARGUMENT, "need 0 <= step < steps and shift > 0");
   std::vector<char> uskip;
-  int rc = check_step_args(m, x, text_c, text_u, n_txt, height, width, cfg, uncond_skip_layers, n_skip, &uskip);
+  int rc = check_step_args(m, x, text_c, n_txt_c, text_u, n_txt_u, height, width, cfg, uncond_skip_layers, n_skip,
+                           &uskip);
   if (rc) return rc;
   if (!slg_on(step, steps, slg_start, slg_stop)) std::fill(uskip.begin(), uskip.end(), 0);
   std::vector<float> sig;
@@ -711,19 +758,20 @@ int moss_denoise_step(moss_model* m, float* x, const float* text_c, const float*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   rc = compute_modulation(m, &sig[step], 1, s);
   if (rc) return rc;
-  return step_impl(m, x, text_c, text_u, n_txt, height, width, sig[step], sig[step + 1], cfg, uskip, m->mod, s);
+  return step_impl(m, x, text_c, n_txt_c, text_u, n_txt_u, height, width, sig[step], sig[step + 1], cfg, uskip,
+                   m->mod, s);
 }
 
 int moss_sample(moss_model* m, int steps, float cfg, double shift, uint64_t seed, const int* uncond_skip_layers,
-                int n_skip, double slg_start, double slg_stop, const float* text_c, const float* text_u, int n_txt,
-                int height, int width, float* latent_out, void* stream) {
+                int n_skip, double slg_start, double slg_stop, const float* text_c, int n_txt_c, const float* text_u,
+                int n_txt_u, int height, int width, float* latent_out, void* stream) {
   g_last_error.clear();
   if (!m) return fail(MOSS_ERR_INVALID_ARGUMENT, "model is NULL");
   if (steps < 1 || steps > m->cfg.max_steps || !(shift > 0.0))
     return fail(MOSS_ERR_INVALID_ARGUMENT, "need 1 <= steps <= max_steps and shift > 0");
   std::vector<char> uskip;
-  int rc = check_step_args(m, latent_out, text_c, text_u, n_txt, height, width, cfg, uncond_skip_layers, n_skip,
-                           &uskip);
+  int rc = check_step_args(m, latent_out, text_c, n_txt_c, text_u, n_txt_u, height, width, cfg, uncond_skip_layers,
+                           n_skip, &uskip);
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t n = static_cast<int64_t>(height / 8) * (width / 8) * 32;
@@ -735,8 +783,8 @@ int moss_sample(moss_model* m, int steps, float cfg, double shift, uint64_t seed
   const std::vector<char> none(m->cfg.layers, 0);
   for (int i = 0; i < steps; ++i) {
     const bool on = slg_on(i, steps, slg_start, slg_stop);
-    rc = step_impl(m, latent_out, text_c, text_u, n_txt, height, width, sig[i], sig[i + 1], cfg, on ? uskip : none,
-                   m->mod + static_cast<int64_t>(i) * m->mod_stride, s);
+    rc = step_impl(m, latent_out, text_c, n_txt_c, text_u, n_txt_u, height, width, sig[i], sig[i + 1], cfg,
+                   on ? uskip : none, m->mod + static_cast<int64_t>(i) * m->mod_stride, s);
     if (rc) return rc;
   }
   return MOSS_OK;

@@ -155,6 +155,12 @@ __device__ __forceinline__ void epi_resid_tma(const EpiParams& ep, const CUtenso
   }
 }
 
+// Token index (within its branch) of a row of the packed [branch; tokens] activations.
+__device__ __forceinline__ int token_of_row(const EpiParams& ep, int row) {
+  if (ep.split_rows > 0) return row >= ep.split_rows ? row - ep.split_rows : row;
+  return row % ep.n_tok;
+}
+
 // The RoPE table is pair-major ([64][n_tok]): for a fixed pair the 32 lanes (consecutive
 // tokens) read one contiguous segment.
 constexpr int kRopePrefetch = 16;  // rotation pairs read before the accumulator is ready
@@ -165,9 +171,9 @@ struct RopePrefetch {
 __device__ __forceinline__ void qkv_prefetch(const EpiParams& ep, int row, int nb, int half, RopePrefetch& pf) {
   const int col = nb * 256 + half * 128;
   if (col < 2 * ep.hidden && col < ep.N) {
-    const float2* rope = ep.rope + row % ep.n_tok;
+    const float2* rope = ep.rope + token_of_row(ep, row);
 #pragma unroll
-    for (int i = 0; i < kRopePrefetch; ++i) pf.cs[i] = __ldg(rope + static_cast<int64_t>(i) * ep.n_tok);
+    for (int i = 0; i < kRopePrefetch; ++i) pf.cs[i] = __ldg(rope + static_cast<int64_t>(i) * ep.rope_stride);
   }
 }
 
@@ -190,13 +196,13 @@ __device__ __forceinline__ void epi_qkv(const EpiParams& ep, uint32_t tb, int ro
     }
     const float rinv = rsqrtf(((ss[0] + ss[1]) + (ss[2] + ss[3])) * (1.0f / 128.0f) + ep.eps);
     const float* gain = region == 0 ? ep.q_gain : ep.k_gain;
-    const float2* rope = ep.rope + row % ep.n_tok;
+    const float2* rope = ep.rope + token_of_row(ep, row);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       float2 cs[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        cs[i] = c * 16 + i < kRopePrefetch ? pf.cs[c * 16 + i] : __ldg(rope + static_cast<int64_t>(c * 16 + i) * ep.n_tok);
+        cs[i] = c * 16 + i < kRopePrefetch ? pf.cs[c * 16 + i] : __ldg(rope + static_cast<int64_t>(c * 16 + i) * ep.rope_stride);
       float v[32];
       tmem_ld32f(th + c * 32, v);
       const float4* g4 = reinterpret_cast<const float4*>(gain + c * 32);

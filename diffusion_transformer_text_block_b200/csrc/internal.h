@@ -34,8 +34,11 @@ struct EpiParams {
   const bf16* bias = nullptr;        // kEpiEmbed, kEpiOut: [N]
   const float* q_gain = nullptr;     // kEpiQkv: [128]
   const float* k_gain = nullptr;     // kEpiQkv: [128]
-  const float2* rope = nullptr;      // kEpiQkv: [64, n_tok] (cos, sin), pair-major
-  int n_tok = 0;                     // tokens per branch
+  const float2* rope = nullptr;      // kEpiQkv: [64, rope_stride] (cos, sin), pair-major
+  int rope_stride = 0;               // kEpiQkv: tokens per pair row of the RoPE table
+  int n_tok = 0;                     // tokens per branch (of the first branch when split_rows > 0)
+  int split_rows = 0;                // kEpiQkv, two branches of different lengths: rows >= split_rows
+                                     // belong to the second branch (token = row - split_rows)
   int hidden = 0;                    // D
   int n_branch = 0;                  // kEpiEmbed: branches written
   int n_img = 0, grid_w = 0, lat_h8 = 0, lat_w8 = 0;  // kEpiOut

@@ -194,21 +194,24 @@ int moss_init_noise(float* x, int64_t n, uint64_t seed, void* stream);
  * (text_c) and, when cfg != 1, of the unconditional branch (text_u) skipping
  * uncond_skip_layers inside the [slg_start, slg_stop] window; then the CFG + Euler update
  * of `x` in place.  cfg == 1 runs no unconditional pass ([INV] Generation settings).
- *   x: device FP32 [height/8, width/8, 32];  text_c, text_u: device FP32 [n_txt, D]
+ * The two prompts may differ in length (the default negative prompt is empty); each branch
+ * attends over its own tokens, without padding ([SGL-MOSS] 5. Batching).
+ *   x: device FP32 [height/8, width/8, 32]
+ *   text_c: device FP32 [n_txt_c, D];  text_u: device FP32 [n_txt_u, D] (unused when cfg == 1)
  *   uncond_skip_layers: host int [n_skip] in 0..L-1.
- * Errors: as moss_dit_forward. */
-int moss_denoise_step(moss_model* m, float* x, const float* text_c, const float* text_u,
-                      int n_txt, int height, int width, int step, int steps, float cfg,
-                      double shift, const int* uncond_skip_layers, int n_skip,
-                      double slg_start, double slg_stop, void* stream);
+ * Errors: as moss_dit_forward; each branch's image + text tokens must fit max_tokens. */
+int moss_denoise_step(moss_model* m, float* x, const float* text_c, int n_txt_c, const float* text_u, int n_txt_u,
+                      int height, int width, int step, int steps, float cfg, double shift,
+                      const int* uncond_skip_layers, int n_skip, double slg_start, double slg_stop, void* stream);
 
 /* The full sampling loop ([SGL-MOSS] 3 defaults: 50 steps, shift 5, CFG 3, empty negative,
  * uncond layer 22 skipped in slg 0.01..1.0): noise from `seed`, then `steps` calls of the
- * denoising step.  latent_out: device FP32 [height/8, width/8, 32] (also the working
- * buffer).  steps <= max_steps of the model's configuration. */
+ * denoising step.  Prompt arguments as for moss_denoise_step.  latent_out: device FP32
+ * [height/8, width/8, 32] (also the working buffer).  steps <= max_steps of the model's
+ * configuration. */
 int moss_sample(moss_model* m, int steps, float cfg, double shift, uint64_t seed,
                 const int* uncond_skip_layers, int n_skip, double slg_start, double slg_stop,
-                const float* text_c, const float* text_u, int n_txt, int height, int width,
+                const float* text_c, int n_txt_c, const float* text_u, int n_txt_u, int height, int width,
                 float* latent_out, void* stream);
 
 /* ------------------------------------------------------------------------------------ */

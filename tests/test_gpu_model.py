@@ -240,3 +240,39 @@ def test_full_denoise_step_matches_manual_cfg(full_model):
     moss.cfg_euler_step(ref, v[0].contiguous(), v[1].contiguous(), 3.0, float(sig[1]), float(sig[2]))
     assert torch.equal(x, ref)
     assert_no_device_error()
+
+
+@pytest.mark.parametrize("n_u", [5, 0])
+def test_sample_tiny_short_negative_prompt(n_u):
+    """Branches of different text lengths (n_u = 0: the empty negative prompt): the tiny
+    4-step run against the oracle, which runs each branch on its own tokens."""
+    model, wg, wn = make_model(TINY, 65, max_tokens=32, max_latent_hw=64, max_steps=4)
+    tc = make_text(1, 16, TINY.hidden, 66)[0]
+    tu = make_text(1, max(n_u, 1), TINY.hidden, 67)[0][:n_u].contiguous()
+    out = model.sample(tc.cuda(), tu.cuda(), 64, 64, steps=4, cfg=3.0, shift=5.0, seed=3,
+                       uncond_skip_layers=[1], slg_start=0.01, slg_stop=1.0)
+    torch.cuda.synchronize()
+    ref = o.sample(wn, TINY.heads, 64, 64, tc.double().numpy(), tu.double().numpy(), steps=4, cfg=3.0, shift=5.0,
+                   seed=3, uncond_skip_layers=(1,), slg_start=0.01, slg_stop=1.0)
+    assert psnr(ref, out.cpu().numpy()) >= 40.0
+    model.close()
+    assert_no_device_error()
+
+
+def test_full_denoise_step_short_negative_prompt(full_model):
+    """1024^2 step with a 512-token prompt and a 77-token negative prompt, packed back to back,
+    equals the two branches run one at a time followed by the CFG + Euler update."""
+    from synth import FULL
+    model, w = full_model
+    x0 = make_latent(128, 128, 21, device="cuda")
+    tc = make_text(1, 512, FULL.hidden, 22, device="cuda")[0].contiguous()
+    tu = make_text(1, 77, FULL.hidden, 23, device="cuda")[0].contiguous()
+    x = x0.clone()
+    model.denoise_step(x, tc, tu, 1024, 1024, 3, 50, 3.0, 5.0, [22], 0.01, 1.0)
+    sig = o.sigma_schedule(50, 5.0)
+    vc = model.forward(x0, tc[None], 1024, 1024, float(sig[3]), skip_layers=[[]]).clone()
+    vu = model.forward(x0, tu[None], 1024, 1024, float(sig[3]), skip_layers=[[22]]).clone()
+    ref = x0.clone()
+    moss.cfg_euler_step(ref, vc[0].contiguous(), vu[0].contiguous(), 3.0, float(sig[3]), float(sig[4]))
+    assert rel_l2(x.cpu().numpy(), ref.cpu().numpy()) <= 1e-6
+    assert_no_device_error()
