@@ -5,20 +5,29 @@
 // (MossInfer integration guide, What works: exact attention; windpaint.ai MOSS-Image specs:
 // 24 heads of 128, image and text tokens in one sequence.)
 //
-// One CTA per (128-query tile, head, branch); two CTAs share an SM.  Keys are taken 64 at a
-// time.  TMEM (256 columns per CTA): S buffers 0 and 1 (64 columns each, FP32) and O (128).
-// Per CTA (192 threads):
-//   warp 0      TMA: the Q tile once, then K_j and V_j (64 keys x 128 dims, two 64-column
-//               boxes with 128-byte swizzle) into two-slot rings.
-//   warp 1      one thread issues, in this order, S_0, S_1, PV_0, S_2, PV_1, ...:
-//               S_j = Q K_j^T into S buffer j%2 (operands in shared memory) and
-//               O += P_j V_j (P_j from TMEM, V_j from shared memory as an MN-major operand).
-//               S_j+1 is computed while the softmax warps work on S_j.  S_j+2 is issued
-//               right after PV_j without waiting for it: MMAs from one thread run in order.
-//   warps 2..5  softmax, one query row per thread: online softmax in the log2 domain, P_j as
-//               BF16 over the first 32 columns of its S buffer, lazy rescale of O (only when
-//               the running maximum grows by more than 2^8, after waiting for the PV product
-//               in flight).  At the end O / l is stored as BF16.
+// One CTA per SM and per (256-query block, head, branch): two 128-query tiles A and B share
+// every K/V tile of 128 keys.  TMEM (512 columns): S_A, S_B (FP32 scores, 128 columns each;
+// P as BF16 pairs over the first 64 columns of its S) and O_A, O_B (FP32, 128 each).
+// Per CTA (384 threads, three warpgroups):
+//   warp 0      TMA: Q_A and Q_B once, then K_j and V_j (128 keys x 128 dims, four 64x64 boxes
+//               with 128-byte swizzle) into two-slot rings.
+//   warp 1      one thread issues S_A(0), S_B(0), then per key tile j:
+//               PV_A(j) in two halves of 64 keys, S_A(j+1), PV_B(j) likewise, S_B(j+1), so
+//               the tensor pipe works for one tile while the other tile's softmax runs.  The
+//               first half of PV_t(j) starts as soon as the softmax has written the first
+//               half of P_t(j).  S_t(j+1) overwrites the columns PV_t(j) reads P_t(j) from;
+//               tcgen05.mma operations issued by one thread execute in issue order, so no
+//               wait is needed between them.
+//   warps 2, 3  idle (they only lend their registers, below).
+//   warps 4..7  softmax of tile A, warps 8..11 of tile B; one query row per thread: the row
+//               of 128 scores in one TMEM load, online softmax in the log2 domain with a lazy
+//               rescale of O (only when the running maximum grows by more than 2^8).  When
+//               S_t(j) is complete, the commit that signalled it also covers PV_t(j-1), so
+//               O_t is stable for the rescale.  At the end O / l is stored as BF16.
+// Registers: the kernel is launched at 168 per thread (384 x 168 = 64512); warps 0..3 give
+// theirs down to 80 and the softmax warpgroups take 208 (128 x 80 + 256 x 208 = 63488), enough
+// for a row of 128 scores plus the packed P without spilling.  The launcher checks the compiled
+// register count against that sum before the first launch.
 // Keys past the sequence end (the TMA fills them with zeros) are masked to -inf.
 #include "common.cuh"
 #include "internal.h"
@@ -27,41 +36,105 @@ namespace moss {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kQTile = 128;                     // queries per CTA
-constexpr int kKTile = 64;                      // keys per step
+constexpr int kThreads = 384;
+constexpr int kRegsLow = 80;    // warps 0..3 after setmaxnreg.dec
+constexpr int kRegsHigh = 208;  // warps 4..11 after setmaxnreg.inc
+constexpr int kQTile = 128;                     // queries per tile (two tiles per CTA)
+constexpr int kKTile = 128;                     // keys per step
 constexpr int kBox = 64 * 128;                  // one TMA box: 64 rows x 64 BF16 columns
-constexpr int kQBytes = 4 * kBox;               // Q: 128 rows x 128 dims
-constexpr int kKVBytes = 2 * kBox;              // K_j or V_j: 64 rows x 128 dims
-constexpr int kSmemBytes = kQBytes + 4 * kKVBytes + 1024 + 256;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kTileBytes = 4 * kBox;            // 128 rows x 128 dims
+constexpr int kSmemBytes = 2 * kTileBytes + 4 * kTileBytes + 1024 + 256;  // Q_A, Q_B, K x2, V x2
+constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-__global__ void __launch_bounds__(kThreads, 2)
+// Load a 128-row x 128-dim tile as four 64x64 boxes: dims half h, rows r at h*2*kBox + r*kBox,
+// giving for each dims half 128 rows of 128 bytes (the K-major 128-byte-swizzle layout).
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int x, int y, int b) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) tma_load_3d(dst + h * 2 * kBox + r * kBox, tm, bar, x + 64 * h, y + 64 * r, b);
+}
+
+// Packed FP32 pairs: one instruction performs the operation on both halves.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// MMA issue with each shared-memory descriptor given as its low word (start address and
+// leading byte offset); the high word (stride 1024 bytes, version 1, 128-byte swizzle) is the
+// same for every operand here and is joined inside the instruction's asm.  Keeping 32-bit
+// values lets the issuing thread run within its small register budget.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 ad, {%1, %5};\n\t"
+      "mov.b64 bd, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kDescHi)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 bd, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kDescHi)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm, bf16* __restrict__ out, int n_tok, int heads, int hidden,
                 float scale_log2, unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // Q halves (dims 0..63, 64..127) are 128 rows x 128 B each: rows 0..63 then 64..127.
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + kQBytes;                  // 2 slots
-  uint8_t* sV = smem + kQBytes + 2 * kKVBytes;   // 2 slots
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kQBytes + 4 * kKVBytes);
+  uint8_t* sQ = smem;                        // [2] tiles A, B
+  uint8_t* sK = smem + 2 * kTileBytes;       // [2] slots
+  uint8_t* sV = smem + 4 * kTileBytes;       // [2] slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * kTileBytes);
   uint64_t* b_q = bars + 0;
   uint64_t* b_kfull = bars + 1;   // [2]
   uint64_t* b_kempty = bars + 3;  // [2]
   uint64_t* b_vfull = bars + 5;   // [2]
   uint64_t* b_vempty = bars + 7;  // [2]
-  uint64_t* b_s = bars + 9;       // [2] S_j complete, per S buffer
-  uint64_t* b_p = bars + 11;      // [2] P_j written, per S buffer
-  uint64_t* b_o = bars + 13;      // PV_j complete (one phase per j)
-  uint64_t* b_drain = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* b_s = bars + 9;       // [2] S_t(j) complete (tile t), one phase per j
+  uint64_t* b_p = bars + 11;      // [2][2] half h of P_t(j) written (index 2 t + h), one phase per j
+  uint64_t* b_done = bars + 15;   // every MMA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * kQTile;
+  const int q0 = blockIdx.x * 2 * kQTile;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int nkv = (n_tok + kKTile - 1) / kKTile;
@@ -74,10 +147,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&b_vfull[i], 1);
       mbar_init(&b_vempty[i], 1);
       mbar_init(&b_s[i], 1);
-      mbar_init(&b_p[i], 4);
     }
-    mbar_init(b_o, 1);
-    mbar_init(b_drain, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&b_p[i], 4);
+    mbar_init(b_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -90,29 +162,29 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem + 128;  // O (FP32); S buffer i at tmem + 64 i
+  // S_t at tmem + 128 t, O_t at tmem + 256 + 128 t.
 
+  // Each warpgroup's role code sits inside the branch that sets its register count.
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0) {
     if (lane == 0) {
       const int xq = h * 128, xk = hidden + h * 128, xv = 2 * hidden + h * 128;
       int k_armed[2] = {-1, -1}, v_armed[2] = {-1, -1};  // parity of the last armed phase
-      mbar_arrive_expect_tx(b_q, kQBytes);
-      for (int half = 0; half < 2; ++half)
-        for (int r = 0; r < 2; ++r)
-          tma_load_3d(sQ + half * 2 * kBox + r * kBox, &tm, b_q, xq + 64 * half, q0 + 64 * r, b);
+      mbar_arrive_expect_tx(b_q, 2 * kTileBytes);
+      load_tile(sQ, &tm, b_q, xq, q0, b);
+      load_tile(sQ + kTileBytes, &tm, b_q, xq, q0 + kQTile, b);
       for (int j = 0; j < nkv; ++j) {
         const int slot = j & 1;
-        const uint32_t use = (j >> 1) & 1;  // this slot's use count parity
+        const uint32_t use = (j >> 1) & 1;
         if (j >= 2 && !mbar_wait(&b_kempty[slot], use ^ 1, err, kErrAttnProducer, abort_flag)) break;
         k_armed[slot] = static_cast<int>(use);
-        mbar_arrive_expect_tx(&b_kfull[slot], kKVBytes);
-        tma_load_3d(sK + slot * kKVBytes, &tm, &b_kfull[slot], xk, j * kKTile, b);
-        tma_load_3d(sK + slot * kKVBytes + kBox, &tm, &b_kfull[slot], xk + 64, j * kKTile, b);
+        mbar_arrive_expect_tx(&b_kfull[slot], kTileBytes);
+        load_tile(sK + slot * kTileBytes, &tm, &b_kfull[slot], xk, j * kKTile, b);
         if (j >= 2 && !mbar_wait(&b_vempty[slot], use ^ 1, err, kErrAttnProducer, abort_flag)) break;
         v_armed[slot] = static_cast<int>(use);
-        mbar_arrive_expect_tx(&b_vfull[slot], kKVBytes);
-        tma_load_3d(sV + slot * kKVBytes, &tm, &b_vfull[slot], xv, j * kKTile, b);
-        tma_load_3d(sV + slot * kKVBytes + kBox, &tm, &b_vfull[slot], xv + 64, j * kKTile, b);
+        mbar_arrive_expect_tx(&b_vfull[slot], kTileBytes);
+        load_tile(sV + slot * kTileBytes, &tm, &b_vfull[slot], xv, j * kKTile, b);
       }
       // Before the CTA may exit, every load issued must have landed (bounded wait).
       const uint64_t t0 = globaltimer_ns();
@@ -132,64 +204,93 @@ __global__ void __launch_bounds__(kThreads, 2)
       constexpr uint32_t kIdescS = idesc_bf16(128, kKTile, false);
       constexpr uint32_t kIdescO = idesc_bf16(128, 128, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      bool ok = mbar_wait(b_q, 0, err, kErrAttnMma, abort_flag);
-      // PV_{j-1}: O += P_{j-1} V_{j-1}
-      auto issue_pv = [&](int jj) -> bool {
-        const int slot = jj & 1;
-        const uint32_t use = (jj >> 1) & 1;
-        if (!mbar_wait(&b_p[slot], use, err, kErrAttnMma, abort_flag)) return false;
-        if (!mbar_wait(&b_vfull[slot], use, err, kErrAttnMma, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t tP = tmem + 64 * slot;
-        const uint32_t vs = v_addr + slot * kKVBytes;
-#pragma unroll
-        for (int k = 0; k < kKTile / 16; ++k)  // keys in steps of 16: P columns advance by 8 words
-          mma_ts(tO, tP + k * 8, sdesc_sw128(vs + k * 16 * 128, kBox, 1024), kIdescO, (jj > 0 || k > 0) ? 1u : 0u);
-        tc_commit(b_o);
-        tc_commit(&b_vempty[slot]);
-        return true;
-      };
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int slot = j & 1;
-        const uint32_t use = (j >> 1) & 1;
-        // S_j reuses the S buffer whose P_{j-2} the PV_{j-2} product reads.  That product
-        // was issued earlier by this thread, and tcgen05.mma operations issued by one thread
-        // execute in issue order, so it has read P_{j-2} before S_j is written: no wait.
-        if (!mbar_wait(&b_kfull[slot], use, err, kErrAttnMma, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t ks = k_addr + slot * kKVBytes;
+      // S_t(j) = Q_t K_j^T into S_t.
+      auto issue_s = [&](int t, int j) {
+        const uint32_t qs = q_addr + t * kTileBytes;
+        const uint32_t ks = k_addr + (j & 1) * kTileBytes;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // head dim in steps of 16
-          const uint32_t qoff = (k >> 2) * 2 * kBox + (k & 3) * 32;
-          const uint32_t koff = (k >> 2) * kBox + (k & 3) * 32;
-          mma_ss(tmem + 64 * slot, sdesc_sw128(q_addr + qoff, 16, 1024), sdesc_sw128(ks + koff, 16, 1024), kIdescS,
-                 k > 0 ? 1u : 0u);
+          const uint32_t off = (k >> 2) * 2 * kBox + (k & 3) * 32;
+          mma_ss_lo(tmem + 128 * t, desc_lo(qs + off, 16), desc_lo(ks + off, 16), kIdescS, k > 0 ? 1u : 0u);
         }
-        tc_commit(&b_s[slot]);
-        tc_commit(&b_kempty[slot]);
-        if (j >= 1 && !issue_pv(j - 1)) {
+        tc_commit(&b_s[t]);
+      };
+      // O_t += P_t(j) V_j over keys 64 h .. 64 h + 63, P from columns 32 h .. 32 h + 31 of S_t.
+      auto issue_pv = [&](int t, int j, int h) {
+        const uint32_t vs = v_addr + (j & 1) * kTileBytes;
+#pragma unroll
+        for (int k = 4 * h; k < 4 * h + 4; ++k)  // keys in steps of 16: P columns advance by 8 words
+          mma_ts_lo(tmem + 256 + 128 * t, tmem + 128 * t + k * 8, desc_lo(vs + k * 16 * 128, 2 * kBox), kIdescO,
+                    (j > 0 || k > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(b_q, 0, err, kErrAttnMma, abort_flag) &&
+                mbar_wait(&b_kfull[0], 0, err, kErrAttnMma, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        tc_commit(&b_kempty[0]);
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const uint32_t use = (j >> 1) & 1;
+        const bool more = j + 1 < nkv;
+        const int nslot = (j + 1) & 1;
+        const uint32_t nuse = ((j + 1) >> 1) & 1;
+        // tile A: the operands that are ready first, then the two halves of P_A(j)
+        if (!mbar_wait(&b_vfull[j & 1], use, err, kErrAttnMma, abort_flag) ||
+            (more && !mbar_wait(&b_kfull[nslot], nuse, err, kErrAttnMma, abort_flag)) ||
+            !mbar_wait(&b_p[0], j & 1, err, kErrAttnMma, abort_flag)) {
           ok = false;
           break;
         }
+        tc_fence_after();
+        issue_pv(0, j, 0);
+        if (!mbar_wait(&b_p[1], j & 1, err, kErrAttnMma, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(0, j, 1);
+        if (more) issue_s(0, j + 1);
+        // tile B
+        if (!mbar_wait(&b_p[2], j & 1, err, kErrAttnMma, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(1, j, 0);
+        if (!mbar_wait(&b_p[3], j & 1, err, kErrAttnMma, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(1, j, 1);
+        tc_commit(&b_vempty[j & 1]);
+        if (more) {
+          issue_s(1, j + 1);
+          tc_commit(&b_kempty[nslot]);
+        }
       }
-      if (ok) issue_pv(nkv - 1);
-      tc_commit(b_drain);
+      tc_commit(b_done);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(smem_u32(b_drain), 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      while (!mbar_try_wait(smem_u32(b_done), 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
     }
+  }
   } else {
-    const int quad = warp & 3;
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+  {
+    const int t = (warp - 4) >> 2;   // query tile: 0 = A (warps 4..7), 1 = B (warps 8..11)
+    const int quad = warp & 3;       // TMEM lane quadrant
     const int r = quad * 32 + lane;  // query row within the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + 128 * t + lane_off;
+    const uint32_t tO = tmem + 256 + 128 * t + lane_off;
     float m_run = -INFINITY;  // running maximum, log2 units (possibly stale by < 2^8)
     float l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int slot = j & 1;
-      const uint32_t use = (j >> 1) & 1;
-      const uint32_t tS = tmem + 64 * slot + lane_off;
-      ok = mbar_wait(&b_s[slot], use, err, kErrAttnSoftmax, abort_flag);
+      ok = mbar_wait(&b_s[t], j & 1, err, kErrAttnSoftmax, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {  // warp-uniform: TMEM accesses are .sync.aligned
         ok = false;
         break;
@@ -197,17 +298,19 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_after();
       const int kvalid = n_tok - j * kKTile;  // keys of this step inside the sequence
       const bool full = kvalid >= kKTile;     // warp-uniform
-      uint32_t sr[64];
-      tmem_ld64(tS, sr);
+      // The whole row of 128 scores in one TMEM load.
+      uint32_t sr[128];
+      tmem_ld128(tS, sr);
       float mxp[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) mxp[a] = -INFINITY;
       if (full) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) mxp[i & 7] = fmaxf(mxp[i & 7], __uint_as_float(sr[i]));
+        for (int i = 0; i < 64; ++i)
+          mxp[i & 7] = max3(mxp[i & 7], __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
       } else {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < 128; ++i)
           if (i < kvalid) mxp[i & 7] = fmaxf(mxp[i & 7], __uint_as_float(sr[i]));
       }
       const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
@@ -217,60 +320,69 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float m_new = grow ? mx : m_run;
       const float factor = grow ? exp2_approx(m_run - m_new) : 1.0f;  // 0 on the first step
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O may still be accumulating PV_{j-1}: wait for it before rescaling.
-        ok = mbar_wait(b_o, (j - 1) & 1, err, kErrAttnSoftmax, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        // PV_t(j-1) was issued before S_t(j) and covered by its commit: O_t is stable.
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO + lane_off + c * 32, o);
+          tmem_ld32(tO + c * 32, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-          tmem_st32(tO + lane_off + c * 32, o);
+          tmem_st32(tO + c * 32, o);
         }
       }
       m_run = m_new;
-      float sump[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
-      if (full) {
+      // Exponentials; P_t(j) over the first 64 columns of S_t, in two 32-column halves, each
+      // signalled to the MMA thread as soon as it is stored.  Row sums in packed pairs.
+      const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
+      const uint64_t negm2 = f2_pack(-m_run, -m_run);
+      uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = exp2_approx(fmaf(__uint_as_float(sr[2 * i]), scale_log2, -m_run));
-          const float p1 = exp2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), scale_log2, -m_run));
-          sump[i & 3] += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-      } else {
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[32];
+        if (full) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = 2 * i < kvalid ? exp2_approx(fmaf(__uint_as_float(sr[2 * i]), scale_log2, -m_run)) : 0.f;
-          const float p1 =
-              2 * i + 1 < kvalid ? exp2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), scale_log2, -m_run)) : 0.f;
-          sump[i & 3] += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 32; ++i) {
+            float x0, x1, p0, p1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[64 * c + 2 * i]), __uint_as_float(sr[64 * c + 2 * i + 1])),
+                             scale2, negm2),
+                      x0, x1);
+            p0 = exp2_approx(x0);
+            p1 = exp2_approx(x1);
+            acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(p0, p1));
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int k0 = 64 * c + 2 * i;
+            const float p0 = k0 < kvalid ? exp2_approx(fmaf(__uint_as_float(sr[k0]), scale_log2, -m_run)) : 0.f;
+            const float p1 =
+                k0 + 1 < kvalid ? exp2_approx(fmaf(__uint_as_float(sr[k0 + 1]), scale_log2, -m_run)) : 0.f;
+            acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(p0, p1));
+            pk[i] = pack_bf16x2(p0, p1);
+          }
         }
+        tmem_st32(tS + 32 * c, pk);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b_p[2 * t + c]);
       }
-      // P_j (BF16 pairs) over the first 32 columns of its S buffer: the A operand of PV_j.
-      tmem_st32(tS, pk);
-      l_run = l_run * factor + ((sump[0] + sump[1]) + (sump[2] + sump[3]));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&b_p[slot]);
+      float a0, a1, b0, b1;
+      f2_unpack(acc2[0], a0, a1);
+      f2_unpack(acc2[1], b0, b1);
+      const float rowsum = (a0 + b0) + (a1 + b1);
+      l_run = l_run * factor + rowsum;
     }
-    if (ok) ok = mbar_wait(b_o, (nkv - 1) & 1, err, kErrAttnSoftmax, abort_flag);
+    if (ok) ok = mbar_wait(b_done, 0, err, kErrAttnSoftmax, abort_flag);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const float inv_l = 1.0f / l_run;
-      const int q = q0 + r;
+      const int q = q0 + kQTile * t + r;
       bf16* dst = out + (static_cast<int64_t>(b) * n_tok + q) * hidden + h * 128;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float v[32];
-        tmem_ld32f(tO + lane_off + c * 32, v);
+        tmem_ld32f(tO + c * 32, v);
         if (q < n_tok) {
           uint4* d = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
@@ -284,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -298,7 +411,17 @@ cudaError_t launch_attention(const bf16* qkv, bf16* o, int batch, int n_tok, int
                              unsigned* err, std::string* emsg) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    // setmaxnreg.inc waits until the registers it asks for are free in the CTA's pool (its
+    // threads x the registers per thread at launch), so a split that does not fit would never
+    // return: refuse to launch unless the compiled count covers it.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * kThreads < 128 * kRegsLow + 256 * kRegsHigh) {
+      if (emsg) *emsg = "attention kernel compiled with too few registers for its register split";
+      return cudaErrorInvalidConfiguration;
+    }
+    e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
@@ -309,7 +432,7 @@ cudaError_t launch_attention(const bf16* qkv, bf16* o, int batch, int n_tok, int
   if (!make_tmap_bf16_3d(&tm, qkv, 3 * static_cast<uint64_t>(hidden), n_tok, batch, 64, kBox / 128, emsg))
     return cudaErrorInvalidValue;
   const float scale_log2 = 1.4426950408889634f / sqrtf(128.0f);
-  dim3 grid((n_tok + kQTile - 1) / kQTile, heads, batch);
+  dim3 grid((n_tok + 2 * kQTile - 1) / (2 * kQTile), heads, batch);
   attn_kernel<<<grid, kThreads, kSmemBytes, s>>>(tm, o, n_tok, heads, hidden, scale_log2, err);
   return cudaGetLastError();
 }
