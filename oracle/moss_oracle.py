@@ -39,6 +39,16 @@ Readings taken where the pages are silent (each repeated where it is used):
       element-group index, Box-Muller on 23-bit uniforms.
   R15 The two CFG branches each attend over their own prompt tokens; their lengths may
       differ and are never padded.
+  R16 CFG truncation X in [0, 1] (1 = off): step i runs the conditional branch alone
+      (v = v_c) when cfg != 1 and i >= X * steps.
+  R17 Step cache: the quantity watched is block 0's output, the residual stream of every
+      branch of the call (image and text rows) right after block 0; its change is
+      sum|o - o_ref| / sum|o_ref| against o_ref, block 0's output at the last full call.
+  R18 A step reuses the cache when a last full call with the same number of branches exists
+      and the change is below the threshold: its stream after the last block is
+      o + (x_L - o_ref) of the last full call (blocks 1..L-1 of that call, as a residual).
+      Otherwise it runs every block and becomes the last full call.  The first step is
+      always a full call.
 """
 from __future__ import annotations
 
@@ -436,6 +446,94 @@ def sample(w: dict, heads: int, height: int, width: int, text_c: np.ndarray, tex
         v_u = dit_forward(x, np.asarray(text_u)[None], t, [skip_u], w, heads, head_dim)[0].astype(F32)
         x = cfg_euler(x, v_c, v_u, cfg, sig[i], sig[i + 1])
     return x
+
+
+# --------------------------------------------------------------------------------------
+# Lossy accelerators, off by default.  [MI] What works (Lossy accelerators) and the opt-in
+# list that follows it; Per-image settings (CFG truncation, Step cache): CFG truncation drops
+# the negative branch from step X*steps on; the step cache (First-Block Cache) reuses blocks
+# 1..L-1 of the last full call while block 0's output changed by less than a threshold.
+# Readings R16-R18.
+# --------------------------------------------------------------------------------------
+def cfg_truncated(step: int, steps: int, cfg_truncation: float) -> bool:
+    """R16: the negative branch is dropped at step `step` (0-based)."""
+    return step >= cfg_truncation * steps
+
+
+def relative_change(outs, refs) -> float:
+    """R17: sum |o - o_ref| / sum |o_ref| over every row of every branch."""
+    num = sum(float(np.sum(np.abs(np.asarray(o, F64) - np.asarray(r, F64)))) for o, r in zip(outs, refs))
+    den = sum(float(np.sum(np.abs(np.asarray(r, F64)))) for r in refs)
+    return num / den
+
+
+def sample_accelerated(w: dict, heads: int, height: int, width: int, text_c: np.ndarray, text_u: np.ndarray,
+                       steps: int = 50, cfg: float = 3.0, shift: float = 5.0, seed: int = 42,
+                       uncond_skip_layers=(22,), slg_start: float = 0.01, slg_stop: float = 1.0,
+                       cfg_truncation: float = 1.0, step_cache_threshold: float = 0.0, decisions=None,
+                       head_dim: int = 128, x0: np.ndarray | None = None):
+    """The sampler of `sample` with CFG truncation (R16) and the step cache (R17, R18).
+
+    step_cache_threshold <= 0 turns the cache off.  `decisions`, when given, replaces the
+    threshold test of each step with decisions[i] (a step without a comparable full call
+    still runs in full): a caller that already took the decisions in another precision
+    replays them.  Returns (x, cached, change): the final latent, per step whether it reused
+    the cache, and the block-0 change measured at that step (NaN when there was nothing to
+    compare with).
+    """
+    ok, msg = validate_size(height, width)
+    if not ok:
+        raise ValueError(msg)
+    h8, w8 = height // 8, width // 8
+    gh, gw = h8 // 2, w8 // 2
+    n_img = gh * gw
+    L = w["wqkv"].shape[0]
+    x = gaussian_noise(h8 * w8 * 32, seed).reshape(h8, w8, 32) if x0 is None else np.asarray(x0, F32).copy()
+    sig = sigma_schedule(steps, shift)
+    use_cache = step_cache_threshold > 0.0 or decisions is not None
+    last = None  # (number of branches, block-0 outputs, residuals of blocks 1..L-1)
+    cached, change = [], []
+    for i in range(steps):
+        t = float(sig[i])
+        two = cfg != 1.0 and not cfg_truncated(i, steps, cfg_truncation)
+        texts = [np.asarray(text_c, F64), np.asarray(text_u, F64)] if two else [np.asarray(text_c, F64)]
+        skip_u = tuple(uncond_skip_layers) if slg_active(i, steps, slg_start, slg_stop) else ()
+        skips = [(), skip_u] if two else [()]
+        c = conditioning(t, w)
+        mods = [block_modulation(c, w["mod_w"][l], w["mod_b"][l]) for l in range(L)]
+        img = patchify(np.asarray(x, F64)) @ w["img_w"].T + w["img_b"]
+        angles = [rope_angles(token_positions(gh, gw, tb.shape[0]), head_dim) for tb in texts]
+        o0 = []
+        for b, tb in enumerate(texts):
+            xb = np.concatenate([img, tb], axis=0)
+            if 0 not in skips[b]:
+                xb = block_forward(xb, layer_weights(w, 0), mods[0], angles[b], heads, head_dim)
+            o0.append(xb)
+        ch = float("nan")
+        reuse = False
+        if use_cache and last is not None and last[0] == len(texts):
+            ch = relative_change(o0, last[1])
+            reuse = bool(decisions[i]) if decisions is not None else ch < step_cache_threshold
+        if reuse:
+            xl = [o0[b] + last[2][b] for b in range(len(texts))]
+        else:
+            xl = []
+            for b in range(len(texts)):
+                xb = o0[b]
+                for l in range(1, L):
+                    if l not in skips[b]:
+                        xb = block_forward(xb, layer_weights(w, l), mods[l], angles[b], heads, head_dim)
+                xl.append(xb)
+            if use_cache:
+                last = (len(texts), o0, [xl[b] - o0[b] for b in range(len(texts))])
+        v = [unpatchify(final_layer(xb[:n_img], c, w), h8, w8, 32).astype(F32) for xb in xl]
+        if two:
+            x = cfg_euler(x, v[0], v[1], cfg, sig[i], sig[i + 1])
+        else:
+            x = euler_update(x, v[0], sig[i], sig[i + 1])
+        cached.append(reuse)
+        change.append(ch)
+    return x, cached, change
 
 
 def psnr(ref: np.ndarray, test: np.ndarray) -> float:
