@@ -256,6 +256,54 @@ def run_op(args):
     return 0
 
 
+def run_accel(args):
+    """Whole 1024^2 images (50 steps, CFG 3, shift 5, uncond skips layer 22 in slg [0.01, 1.0])
+    through moss_sample and moss_sample_ex with the lossy accelerators (CFG truncation, the
+    first-block step cache at the pages' default thresholds 0.02 and 0.03).  Random-init
+    weights: how often the cache engages depends on the weights, so the reuse counts here say
+    nothing about a trained model.  Prints one JSON line: seconds per image (CUDA events around
+    each call) and the number of reused steps."""
+    import torch
+
+    import diffusion_transformer_text_block_b200 as moss
+    from synth import FULL, make_text, make_weights
+
+    w = make_weights(FULL, 2, device="cuda")
+    model = moss.Model(FULL, w, max_tokens=4096 + N_TXT, max_batch=2, max_latent_hw=128 * 128, max_steps=50)
+    tc = make_text(1, N_TXT, FULL.hidden, 100, device="cuda")[0].contiguous()
+    tu = make_text(1, N_TXT, FULL.hidden, 200, device="cuda")[0].contiguous()
+    kw = dict(steps=STEPS_PER_IMAGE, cfg=CFG, shift=SHIFT, seed=42, uncond_skip_layers=SKIP, slg_start=SLG[0],
+              slg_stop=SLG[1])
+    runs = [("plain", None), ("cfg_truncation_0.5", dict(cfg_truncation=0.5)),
+            ("step_cache_0.02", dict(step_cache_threshold=0.02)), ("step_cache_0.03", dict(step_cache_threshold=0.03)),
+            ("both_0.5_0.03", dict(cfg_truncation=0.5, step_cache_threshold=0.03))]
+    model.sample(tc, tu, HEIGHT, WIDTH, **dict(kw, steps=2))  # warm-up
+    torch.cuda.synchronize()
+    out = {"op": "accel", "workload": "1024^2 image, 50 steps, CFG 3, random-init 42-block DiT", "runs": {}}
+    base = None
+    for name, opt in runs:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        if opt is None:
+            model.sample(tc, tu, HEIGHT, WIDTH, **kw)
+            cached, change = [False] * STEPS_PER_IMAGE, []
+        else:
+            _, cached, change = model.sample_accelerated(tc, tu, HEIGHT, WIDTH, **kw, **opt)
+        e1.record()
+        torch.cuda.synchronize()
+        s_img = e0.elapsed_time(e1) / 1e3
+        base = base or s_img
+        rec = {"s_per_image": round(s_img, 3), "speedup": round(base / s_img, 3), "reused_steps": int(sum(cached))}
+        finite = [c for c in change if c == c]
+        if finite:
+            rec["change_min_max"] = [round(min(finite), 5), round(max(finite), 5)]
+        out["runs"][name] = rec
+    out["device_status"] = moss.device_status(clear=True)
+    model.close()
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -264,11 +312,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["block", "attention"], default=None,
-                    help="time one kernel class on the 1024^2 shapes instead of the denoising step")
+    ap.add_argument("--op", choices=["block", "attention", "accel"], default=None,
+                    help="time one kernel class on the 1024^2 shapes instead of the denoising step; "
+                         "'accel' times whole 50-step images with the lossy accelerators")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "accel":
+        return run_accel(args)
     if args.op:
         return run_op(args)
 

@@ -43,6 +43,12 @@ class Weights(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32)] + [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
 
 
+class SampleOptions(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("cfg_truncation", ctypes.c_double),
+                ("step_cache_threshold", ctypes.c_double), ("cached_out", ctypes.POINTER(ctypes.c_int)),
+                ("change_out", ctypes.POINTER(ctypes.c_float))]
+
+
 _lib = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -66,6 +72,9 @@ _SIGS = {
     "moss_init_noise": (_I, [_P, _I64, ctypes.c_uint64, _P]),
     "moss_denoise_step": (_I, [_P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _F, _D, _P, _I, _D, _D, _P]),
     "moss_sample": (_I, [_P, _I, _F, _D, ctypes.c_uint64, _P, _I, _D, _D, _P, _I, _P, _I, _I, _I, _P, _P]),
+    "moss_sample_options_init": (None, [ctypes.POINTER(SampleOptions), ctypes.c_uint32]),
+    "moss_sample_ex": (_I, [_P, _I, _F, _D, ctypes.c_uint64, _P, _I, _D, _D, _P, _I, _P, _I, _I, _I,
+                            ctypes.POINTER(SampleOptions), _P, _P]),
     "moss_device_status": (_I, [_I]),
     "moss_profile_enable": (_I, [_P, _I]),
     "moss_profile_read": (_I, [_P, _I, ctypes.POINTER(_I64), ctypes.POINTER(_D)]),
@@ -317,6 +326,31 @@ class Model:
                                  _ptr(text_u, f, "text_u") if text_u is not None else None, n_u,
                                  height, width, _ptr(out, f, "out"), _stream(stream)))
         return out
+
+    def sample_accelerated(self, text_c, text_u, height: int, width: int, steps: int = 50, cfg: float = 3.0,
+                           shift: float = 5.0, seed: int = 42, uncond_skip_layers: Sequence[int] = (22,),
+                           slg_start: float = 0.01, slg_stop: float = 1.0, cfg_truncation: float = 1.0,
+                           step_cache_threshold: float = 0.0, stream=None, out=None):
+        """moss_sample_ex: returns (latent, cached [steps] list of bool, change [steps] list of float)."""
+        import torch
+        if out is None:
+            out = torch.empty(height // 8, width // 8, 32, device=text_c.device, dtype=torch.float32)
+        arr, n = _skip_array([list(uncond_skip_layers)])
+        f = torch.float32
+        n_u = text_u.shape[0] if text_u is not None else 0
+        opt = SampleOptions()
+        lib().moss_sample_options_init(ctypes.byref(opt), ctypes.sizeof(SampleOptions))
+        opt.cfg_truncation = cfg_truncation
+        opt.step_cache_threshold = step_cache_threshold
+        cached = (ctypes.c_int * steps)()
+        change = (ctypes.c_float * steps)()
+        opt.cached_out = ctypes.cast(cached, ctypes.POINTER(ctypes.c_int))
+        opt.change_out = ctypes.cast(change, ctypes.POINTER(ctypes.c_float))
+        _check(lib().moss_sample_ex(self._h, steps, cfg, shift, seed, arr, n, slg_start, slg_stop,
+                                    _ptr(text_c, f, "text_c"), text_c.shape[0],
+                                    _ptr(text_u, f, "text_u") if text_u is not None else None, n_u,
+                                    height, width, ctypes.byref(opt), _ptr(out, f, "out"), _stream(stream)))
+        return out, [bool(c) for c in cached], [float(c) for c in change]
 
     def modulation(self, t: float, stream=None):
         import torch

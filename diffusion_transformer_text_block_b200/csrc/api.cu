@@ -17,6 +17,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <limits>
 #include <vector>
 
 #include "../../include/moss_dit.h"
@@ -205,6 +206,12 @@ struct moss_model {
   int rope_gh = -1, rope_gw = -1, rope_nt = -1;
   int rope_n = 0;  // tokens of the cached RoPE table (its pair-row stride)
   unsigned* err = nullptr;
+  // first-block step cache (allocated on first use): block 0's output at the last full call,
+  // the residual of blocks 1..L-1 of that call, and the change partial sums
+  float* cache_ref = nullptr;
+  float* cache_res = nullptr;
+  double* chg_dev = nullptr;
+  double* chg_host = nullptr;  // pinned
   // weight descriptors
   std::vector<CUtensorMap> tm_qkv, tm_wo, tm_wg, tm_wu, tm_wd;
   CUtensorMap tm_img, tm_out;
@@ -392,73 +399,104 @@ int block_impl(moss_model* m, int l, float* x, const std::vector<int>& lens, con
 // The DiT for `batch` branches sharing `latent`, branch b with n_txts[b] text tokens (equal
 // lengths for any batch, or two branches of different lengths); the branches' rows are packed
 // back to back in the residual stream.  skip[b][l] != 0: branch b skips layer l.
-int forward_impl(moss_model* m, int batch, const float* latent, const float* const* texts, const int* n_txts,
-                 int height, int width, const float* mod, const std::vector<std::vector<char>>& skip, float* v_out,
-                 cudaStream_t s) {
-  const moss_config& c = m->cfg;
-  const int D = c.hidden, L = c.layers;
-  const int h8 = height / 8, w8 = width / 8, gh = height / 16, gw = width / 16;
-  const int n_img = gh * gw;
-  std::vector<int> lens(batch);
-  std::vector<int64_t> off(batch + 1, 0);
+// Row layout of one call: branch b has lens[b] = n_img + n_txt[b] rows starting at off[b].
+struct CallRows {
+  int batch = 0, n_img = 0, gh = 0, gw = 0, h8 = 0, w8 = 0;
+  std::vector<int> lens;
+  std::vector<int64_t> off;
+};
+
+// Patch embedding of the latent into every branch's image rows and the text states into its
+// text rows of the residual stream m->x.
+int embed_impl(moss_model* m, int batch, const float* latent, const float* const* texts, const int* n_txts,
+               int height, int width, CallRows* rows, cudaStream_t s) {
+  const int D = m->cfg.hidden;
+  CallRows& r = *rows;
+  r.batch = batch;
+  r.h8 = height / 8; r.w8 = width / 8; r.gh = height / 16; r.gw = width / 16;
+  r.n_img = r.gh * r.gw;
+  r.lens.assign(batch, 0);
+  r.off.assign(batch + 1, 0);
   int n_txt_max = 0;
   bool equal = true;
   for (int b = 0; b < batch; ++b) {
-    lens[b] = n_img + n_txts[b];
-    off[b + 1] = off[b] + lens[b];
+    r.lens[b] = r.n_img + n_txts[b];
+    r.off[b + 1] = r.off[b] + r.lens[b];
     n_txt_max = std::max(n_txt_max, n_txts[b]);
     equal = equal && n_txts[b] == n_txts[0];
   }
   if (!equal && batch > 2)
     return fail(MOSS_ERR_UNSUPPORTED, "branches of different text lengths are supported for two branches");
-  int rc = ensure_rope(m, gh, gw, n_txt_max, s);
+  int rc = ensure_rope(m, r.gh, r.gw, n_txt_max, s);
   if (rc) return rc;
 
-  LAUNCH(m, MOSS_K_OTHER, s, launch_patchify(latent, m->patches, h8, w8, s), "patchify");
+  LAUNCH(m, MOSS_K_OTHER, s, launch_patchify(latent, m->patches, r.h8, r.w8, s), "patchify");
   std::string e;
   CUtensorMap tm_p;
-  if (!make_tmap_bf16_2d(&tm_p, m->patches, 128, n_img, kGemmBoxK, kGemmBoxRows, &e)) return fail(MOSS_ERR_CUDA, e);
+  if (!make_tmap_bf16_2d(&tm_p, m->patches, 128, r.n_img, kGemmBoxK, kGemmBoxRows, &e)) return fail(MOSS_ERR_CUDA, e);
   EpiParams pe;
-  pe.M = n_img; pe.N = D; pe.K = 128;
+  pe.M = r.n_img; pe.N = D; pe.K = 128;
   pe.out_f32 = m->x; pe.bias = static_cast<const bf16*>(m->w.img_b);
-  pe.n_tok = lens[0]; pe.n_branch = batch;  // branch b's rows start at b * lens[0] (batch <= 2 if ragged)
+  pe.n_tok = r.lens[0]; pe.n_branch = batch;  // branch b's rows start at b * lens[0] (batch <= 2 if ragged)
   LAUNCH(m, MOSS_K_OTHER, s, launch_gemm(kEpiEmbed, tm_p, m->tm_img, m->tm_img, pe, s, m->err), "patch embed");
   for (int b = 0; b < batch; ++b) {
     if (n_txts[b] == 0) continue;
-    MOSS_CUDA(cudaMemcpyAsync(m->x + (off[b] + n_img) * D, texts[b], sizeof(float) * static_cast<size_t>(n_txts[b]) * D,
-                              cudaMemcpyDeviceToDevice, s),
+    MOSS_CUDA(cudaMemcpyAsync(m->x + (r.off[b] + r.n_img) * D, texts[b],
+                              sizeof(float) * static_cast<size_t>(n_txts[b]) * D, cudaMemcpyDeviceToDevice, s),
               "copy text states");
   }
+  return MOSS_OK;
+}
 
-  for (int l = 0; l < L; ++l) {
+// Blocks l0 .. l1-1 on the residual stream; consecutive branches that run a layer share a call.
+int blocks_impl(moss_model* m, int l0, int l1, const CallRows& r, const float* mod,
+                const std::vector<std::vector<char>>& skip, cudaStream_t s) {
+  const int D = m->cfg.hidden;
+  for (int l = l0; l < l1; ++l) {
     int b = 0;
-    while (b < batch) {
+    while (b < r.batch) {
       if (skip[b][l]) {
         ++b;
         continue;
       }
       int e2 = b;
-      while (e2 < batch && !skip[e2][l]) ++e2;
-      const std::vector<int> run(lens.begin() + b, lens.begin() + e2);
-      rc = block_impl(m, l, m->x + off[b] * D, run, mod + static_cast<int64_t>(l) * 6 * D, s);
+      while (e2 < r.batch && !skip[e2][l]) ++e2;
+      const std::vector<int> run(r.lens.begin() + b, r.lens.begin() + e2);
+      int rc = block_impl(m, l, m->x + r.off[b] * D, run, mod + static_cast<int64_t>(l) * 6 * D, s);
       if (rc) return rc;
       b = e2;
     }
   }
+  return MOSS_OK;
+}
 
+// Final LayerNorm-modulation of the image rows and the output projection into v_out.
+int final_impl(moss_model* m, const CallRows& r, const float* mod, float* v_out, cudaStream_t s) {
+  const int D = m->cfg.hidden, L = m->cfg.layers;
   const float* fmod = mod + static_cast<int64_t>(L) * 6 * D;
-  const int rows = batch * n_img;
+  const int rows = r.batch * r.n_img;
   // Image rows of branch b start at b * lens[0] (equal lengths, or two branches).
-  LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(m->x, fmod, fmod + D, m->h, rows, D, n_img, lens[0], 1e-6f, s),
+  LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(m->x, fmod, fmod + D, m->h, rows, D, r.n_img, r.lens[0], 1e-6f, s),
          "final ln");
+  std::string e;
   CUtensorMap tm_hf;
   if (!make_tmap_bf16_2d(&tm_hf, m->h, D, rows, kGemmBoxK, kGemmBoxRows, &e)) return fail(MOSS_ERR_CUDA, e);
   EpiParams oe;
   oe.M = rows; oe.N = 128; oe.K = D;
   oe.out_f32 = v_out; oe.bias = static_cast<const bf16*>(m->w.out_b);
-  oe.n_img = n_img; oe.grid_w = gw; oe.lat_h8 = h8; oe.lat_w8 = w8;
+  oe.n_img = r.n_img; oe.grid_w = r.gw; oe.lat_h8 = r.h8; oe.lat_w8 = r.w8;
   LAUNCH(m, MOSS_K_OTHER, s, launch_gemm(kEpiOut, tm_hf, m->tm_out, m->tm_out, oe, s, m->err), "output projection");
   return MOSS_OK;
+}
+
+int forward_impl(moss_model* m, int batch, const float* latent, const float* const* texts, const int* n_txts,
+                 int height, int width, const float* mod, const std::vector<std::vector<char>>& skip, float* v_out,
+                 cudaStream_t s) {
+  CallRows r;
+  int rc = embed_impl(m, batch, latent, texts, n_txts, height, width, &r, s);
+  if (!rc) rc = blocks_impl(m, 0, m->cfg.layers, r, mod, skip, s);
+  if (!rc) rc = final_impl(m, r, mod, v_out, s);
+  return rc;
 }
 
 int parse_skips(moss_model* m, int batch, const int* skip_layers, int n_skip, std::vector<std::vector<char>>* out) {
@@ -490,6 +528,90 @@ int step_impl(moss_model* m, float* x, const float* text_c, int n_txt_c, const f
   const float* vu = batch == 2 ? m->v + n : m->v;
   LAUNCH(m, MOSS_K_CFG_EULER, s, launch_cfg_euler(x, m->v, vu, n, batch == 2 ? cfg : 1.0f, sigma, sigma_next, s),
          "cfg euler");
+  return MOSS_OK;
+}
+
+// State of the first-block step cache across the steps of one sampling call.
+struct StepCache {
+  bool have_ref = false;  // a full call has stored its block-0 output and residual
+  int batch = 0;          // its number of branches
+  int64_t n = 0;          // and its residual-stream elements
+};
+
+int ensure_cache_buffers(moss_model* m) {
+  if (m->cache_ref) return MOSS_OK;
+  const size_t bytes = sizeof(float) * static_cast<size_t>(m->rows_cap) * m->cfg.hidden;
+  const size_t pbytes = sizeof(double) * 2 * change_partial_blocks();
+  if (cudaMalloc(&m->cache_ref, bytes) != cudaSuccess || cudaMalloc(&m->cache_res, bytes) != cudaSuccess ||
+      cudaMalloc(&m->chg_dev, pbytes) != cudaSuccess || cudaMallocHost(&m->chg_host, pbytes) != cudaSuccess) {
+    cudaGetLastError();
+    if (m->cache_ref) cudaFree(m->cache_ref);
+    if (m->cache_res) cudaFree(m->cache_res);
+    if (m->chg_dev) cudaFree(m->chg_dev);
+    if (m->chg_host) cudaFreeHost(m->chg_host);
+    m->cache_ref = m->cache_res = nullptr;
+    m->chg_dev = m->chg_host = nullptr;
+    return fail(MOSS_ERR_OOM, "cannot allocate the step-cache buffers");
+  }
+  return MOSS_OK;
+}
+
+// One step of the sampling loop with the lossy accelerators: `two` = run the unconditional
+// branch (false once CFG truncation has dropped it); threshold > 0 = first-block step cache.
+int accel_step_impl(moss_model* m, float* x, const float* text_c, int n_txt_c, const float* text_u, int n_txt_u,
+                    int height, int width, float sigma, float sigma_next, float cfg, bool two,
+                    const std::vector<char>& uskip, const float* mod, double threshold, StepCache* sc, int* cached,
+                    float* change, cudaStream_t s) {
+  const int batch = two ? 2 : 1;
+  const int D = m->cfg.hidden, L = m->cfg.layers;
+  std::vector<std::vector<char>> skips(batch, std::vector<char>(L, 0));
+  if (two) skips[1] = uskip;
+  const float* texts[2] = {text_c, text_u};
+  const int n_txts[2] = {n_txt_c, n_txt_u};
+  CallRows r;
+  int rc = embed_impl(m, batch, x, texts, n_txts, height, width, &r, s);
+  if (!rc) rc = blocks_impl(m, 0, 1, r, mod, skips, s);
+  if (rc) return rc;
+  const int64_t n = r.off[batch] * D;
+  bool reuse = false;
+  double ch = std::numeric_limits<double>::quiet_NaN();
+  if (threshold > 0.0 && sc->have_ref && sc->batch == batch && sc->n == n) {
+    LAUNCH(m, MOSS_K_OTHER, s, launch_change_partials(m->x, m->cache_ref, n, m->chg_dev, s), "step-cache change");
+    const int nb = change_partial_blocks();
+    MOSS_CUDA(cudaMemcpyAsync(m->chg_host, m->chg_dev, sizeof(double) * 2 * nb, cudaMemcpyDeviceToHost, s),
+              "read step-cache change");
+    MOSS_CUDA(cudaStreamSynchronize(s), "wait for step-cache change");
+    double num = 0.0, den = 0.0;
+    for (int i = 0; i < nb; ++i) {
+      num += m->chg_host[2 * i];
+      den += m->chg_host[2 * i + 1];
+    }
+    ch = den > 0.0 ? num / den : (num == 0.0 ? 0.0 : std::numeric_limits<double>::infinity());
+    reuse = ch < threshold;
+  }
+  if (reuse) {
+    LAUNCH(m, MOSS_K_OTHER, s, launch_add_inplace(m->x, m->cache_res, n, s), "step-cache reuse");
+  } else {
+    if (threshold > 0.0)
+      MOSS_CUDA(cudaMemcpyAsync(m->cache_ref, m->x, sizeof(float) * n, cudaMemcpyDeviceToDevice, s),
+                "store block-0 output");
+    rc = blocks_impl(m, 1, L, r, mod, skips, s);
+    if (rc) return rc;
+    if (threshold > 0.0) {
+      LAUNCH(m, MOSS_K_OTHER, s, launch_sub(m->cache_res, m->x, m->cache_ref, n, s), "store block residual");
+      sc->have_ref = true;
+      sc->batch = batch;
+      sc->n = n;
+    }
+  }
+  rc = final_impl(m, r, mod, m->v, s);
+  if (rc) return rc;
+  const int64_t nl = static_cast<int64_t>(height / 8) * (width / 8) * 32;
+  const float* vu = two ? m->v + nl : m->v;
+  LAUNCH(m, MOSS_K_CFG_EULER, s, launch_cfg_euler(x, m->v, vu, nl, two ? cfg : 1.0f, sigma, sigma_next, s),
+         "cfg euler");
+  *cached = reuse ? 1 : 0;
+  *change = static_cast<float>(ch);
   return MOSS_OK;
 }
 
@@ -637,9 +759,11 @@ int moss_model_create(const moss_config* cfg, const moss_weights* w, moss_model*
 void moss_model_free(moss_model* m) {
   if (!m) return;
   cudaDeviceSynchronize();
-  void* bufs[] = {m->x, m->h, m->qkv, m->attn, m->act, m->patches, m->v, m->rope, m->mod, m->sc, m->tvals};
+  void* bufs[] = {m->x,   m->h,  m->qkv,   m->attn,      m->act,      m->patches, m->v,
+                  m->rope, m->mod, m->sc, m->tvals, m->cache_ref, m->cache_res, m->chg_dev};
   for (void* p : bufs)
     if (p) cudaFree(p);
+  if (m->chg_host) cudaFreeHost(m->chg_host);
   for (cudaEvent_t e : m->events) cudaEventDestroy(e);
   delete m;
 }
@@ -786,6 +910,69 @@ int moss_sample(moss_model* m, int steps, float cfg, double shift, uint64_t seed
     rc = step_impl(m, latent_out, text_c, n_txt_c, text_u, n_txt_u, height, width, sig[i], sig[i + 1], cfg,
                    on ? uskip : none, m->mod + static_cast<int64_t>(i) * m->mod_stride, s);
     if (rc) return rc;
+  }
+  return MOSS_OK;
+}
+
+void moss_sample_options_init(moss_sample_options* opt, uint32_t struct_size) {
+  if (!opt || struct_size < sizeof(uint32_t)) return;
+  moss_sample_options d;
+  std::memset(&d, 0, sizeof d);
+  d.cfg_truncation = 1.0;
+  d.step_cache_threshold = 0.0;
+  std::memcpy(opt, &d, std::min<size_t>(struct_size, sizeof d));
+  opt->struct_size = struct_size;
+}
+
+int moss_sample_ex(moss_model* m, int steps, float cfg, double shift, uint64_t seed, const int* uncond_skip_layers,
+                   int n_skip, double slg_start, double slg_stop, const float* text_c, int n_txt_c,
+                   const float* text_u, int n_txt_u, int height, int width, const moss_sample_options* opt_in,
+                   float* latent_out, void* stream) {
+  g_last_error.clear();
+  moss_sample_options opt;
+  moss_sample_options_init(&opt, sizeof opt);
+  if (opt_in) {
+    if (opt_in->struct_size != sizeof(moss_sample_options))
+      return fail(MOSS_ERR_ABI_MISMATCH,
+                  "moss_sample_options.struct_size is not sizeof(moss_sample_options) of this library");
+    opt = *opt_in;
+  }
+  if (!(opt.cfg_truncation >= 0.0 && opt.cfg_truncation <= 1.0))
+    return fail(MOSS_ERR_INVALID_ARGUMENT, "cfg_truncation must lie in [0, 1]");
+  if (!(opt.step_cache_threshold >= 0.0))
+    return fail(MOSS_ERR_INVALID_ARGUMENT, "step_cache_threshold must be >= 0");
+  if (!m) return fail(MOSS_ERR_INVALID_ARGUMENT, "model is NULL");
+  if (steps < 1 || steps > m->cfg.max_steps || !(shift > 0.0))
+    return fail(MOSS_ERR_INVALID_ARGUMENT, "need 1 <= steps <= max_steps and shift > 0");
+  std::vector<char> uskip;
+  int rc = check_step_args(m, latent_out, text_c, n_txt_c, text_u, n_txt_u, height, width, cfg, uncond_skip_layers,
+                           n_skip, &uskip);
+  if (rc) return rc;
+  const double thr = opt.step_cache_threshold;
+  if (thr > 0.0) {
+    rc = ensure_cache_buffers(m);
+    if (rc) return rc;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n = static_cast<int64_t>(height / 8) * (width / 8) * 32;
+  LAUNCH(m, MOSS_K_OTHER, s, launch_noise(latent_out, n, seed, s), "noise");
+  std::vector<float> sig;
+  host_schedule(steps, shift, &sig);
+  rc = compute_modulation(m, sig.data(), steps, s);
+  if (rc) return rc;
+  const std::vector<char> none(m->cfg.layers, 0);
+  StepCache sc;
+  for (int i = 0; i < steps; ++i) {
+    const bool on = slg_on(i, steps, slg_start, slg_stop);
+    const bool two = cfg != 1.0f && !(static_cast<double>(i) >= opt.cfg_truncation * steps);
+    int cached = 0;
+    float change = 0.f;
+    rc = accel_step_impl(m, latent_out, text_c, n_txt_c, text_u, n_txt_u, height, width, sig[i], sig[i + 1], cfg,
+                         two, on ? uskip : none, m->mod + static_cast<int64_t>(i) * m->mod_stride, thr, &sc,
+                         &cached, &change, s);
+    if (rc) return rc;
+    if (opt.cached_out) opt.cached_out[i] = cached;
+    if (opt.change_out) opt.change_out[i] = change;
   }
   return MOSS_OK;
 }

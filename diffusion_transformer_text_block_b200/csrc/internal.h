@@ -101,4 +101,11 @@ cudaError_t launch_rope_table(float2* table, int grid_h, int grid_w, int n_txt, 
 
 cudaError_t launch_patchify(const float* latent, bf16* tokens, int h8, int w8, cudaStream_t s);
 
+// Step cache (first-block cache): per-block FP64 partial sums of |a - ref| and |ref| over n
+// elements into partials[2 * change_partial_blocks()]; x += r; d = a - b.
+int change_partial_blocks();
+cudaError_t launch_change_partials(const float* a, const float* ref, int64_t n, double* partials, cudaStream_t s);
+cudaError_t launch_add_inplace(float* x, const float* r, int64_t n, cudaStream_t s);
+cudaError_t launch_sub(float* d, const float* a, const float* b, int64_t n, cudaStream_t s);
+
 }  // namespace moss

@@ -214,6 +214,42 @@ int moss_sample(moss_model* m, int steps, float cfg, double shift, uint64_t seed
                 const float* text_c, int n_txt_c, const float* text_u, int n_txt_u, int height, int width,
                 float* latent_out, void* stream);
 
+/* Lossy accelerators of the sampling loop, both off by default ([MI] What works: Lossy
+ * accelerators; Per-image settings: CFG truncation, Step cache).  They change the image. */
+typedef struct moss_sample_options {
+  uint32_t struct_size;        /* sizeof(moss_sample_options) as compiled by the caller       */
+  /* CFG truncation, in [0, 1]; 1 (the default) is off.  Step i (0-based) with
+   * i >= cfg_truncation * steps (compared in double) runs the conditional branch alone and
+   * takes v = v_c.  No effect at cfg 1. */
+  double cfg_truncation;
+  /* First-block step cache: > 0 turns it on, 0 (the default) is off.  Each step runs block 0;
+   * its output o (every row of every branch of the call) is compared with o_ref, block 0's
+   * output at the last full call: change = sum|o - o_ref| / sum|o_ref|, summed in FP64.
+   * change < threshold reuses the last full call's blocks 1..layers-1 as a residual
+   * (stream = o + (x_L - o_ref) of that call); otherwise the step runs every block and becomes
+   * the last full call.  The first step, and a step whose number of branches differs from the
+   * last full call's (CFG truncation), always runs in full. */
+  double step_cache_threshold;
+  int* cached_out;    /* optional HOST int [steps]: 1 where the step reused the cache, else 0 */
+  float* change_out;  /* optional HOST float [steps]: the change measured at the step, NaN where
+                         there was no full call to compare with (or the cache is off) */
+} moss_sample_options;
+
+/* Defaults: cfg_truncation = 1, step_cache_threshold = 0, no outputs; struct_size as given. */
+void moss_sample_options_init(moss_sample_options* opt, uint32_t struct_size);
+
+/* moss_sample with the accelerators of `opt` (NULL = defaults, identical to moss_sample).
+ * With the step cache on, the call waits on `stream` once per step (the host reads the change
+ * to choose the step's path) and, on first use, allocates two FP32 buffers of
+ * max_batch x max_tokens x hidden owned by the model (freed by moss_model_free).
+ * Errors: as moss_sample; MOSS_ERR_ABI_MISMATCH when struct_size is not this version's;
+ * MOSS_ERR_INVALID_ARGUMENT for cfg_truncation outside [0, 1] or a negative or NaN threshold;
+ * MOSS_ERR_OOM when the cache buffers cannot be allocated. */
+int moss_sample_ex(moss_model* m, int steps, float cfg, double shift, uint64_t seed,
+                   const int* uncond_skip_layers, int n_skip, double slg_start, double slg_stop,
+                   const float* text_c, int n_txt_c, const float* text_u, int n_txt_u, int height, int width,
+                   const moss_sample_options* opt, float* latent_out, void* stream);
+
 /* ------------------------------------------------------------------------------------ */
 /* Status, profiling and operator-level entry points (used by tests and the benchmark). */
 /* ------------------------------------------------------------------------------------ */

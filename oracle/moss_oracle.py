@@ -39,12 +39,12 @@ Readings taken where the pages are silent (each repeated where it is used):
       element-group index, Box-Muller on 23-bit uniforms.
   R15 The two CFG branches each attend over their own prompt tokens; their lengths may
       differ and are never padded.
-  R16 CFG truncation X in [0, 1] (1 = off): step i runs the conditional branch alone
+  R19 CFG truncation X in [0, 1] (1 = off): step i runs the conditional branch alone
       (v = v_c) when cfg != 1 and i >= X * steps.
-  R17 Step cache: the quantity watched is block 0's output, the residual stream of every
+  R20 Step cache: the quantity watched is block 0's output, the residual stream of every
       branch of the call (image and text rows) right after block 0; its change is
       sum|o - o_ref| / sum|o_ref| against o_ref, block 0's output at the last full call.
-  R18 A step reuses the cache when a last full call with the same number of branches exists
+  R21 A step reuses the cache when a last full call with the same number of branches exists
       and the change is below the threshold: its stream after the last block is
       o + (x_L - o_ref) of the last full call (blocks 1..L-1 of that call, as a residual).
       Otherwise it runs every block and becomes the last full call.  The first step is
@@ -453,15 +453,15 @@ def sample(w: dict, heads: int, height: int, width: int, text_c: np.ndarray, tex
 # list that follows it; Per-image settings (CFG truncation, Step cache): CFG truncation drops
 # the negative branch from step X*steps on; the step cache (First-Block Cache) reuses blocks
 # 1..L-1 of the last full call while block 0's output changed by less than a threshold.
-# Readings R16-R18.
+# Readings R19-R21.
 # --------------------------------------------------------------------------------------
 def cfg_truncated(step: int, steps: int, cfg_truncation: float) -> bool:
-    """R16: the negative branch is dropped at step `step` (0-based)."""
+    """R19: the negative branch is dropped at step `step` (0-based)."""
     return step >= cfg_truncation * steps
 
 
 def relative_change(outs, refs) -> float:
-    """R17: sum |o - o_ref| / sum |o_ref| over every row of every branch."""
+    """R20: sum |o - o_ref| / sum |o_ref| over every row of every branch."""
     num = sum(float(np.sum(np.abs(np.asarray(o, F64) - np.asarray(r, F64)))) for o, r in zip(outs, refs))
     den = sum(float(np.sum(np.abs(np.asarray(r, F64)))) for r in refs)
     return num / den
@@ -472,7 +472,7 @@ def sample_accelerated(w: dict, heads: int, height: int, width: int, text_c: np.
                        uncond_skip_layers=(22,), slg_start: float = 0.01, slg_stop: float = 1.0,
                        cfg_truncation: float = 1.0, step_cache_threshold: float = 0.0, decisions=None,
                        head_dim: int = 128, x0: np.ndarray | None = None):
-    """The sampler of `sample` with CFG truncation (R16) and the step cache (R17, R18).
+    """The sampler of `sample` with CFG truncation (R19) and the step cache (R20, R21).
 
     step_cache_threshold <= 0 turns the cache off.  `decisions`, when given, replaces the
     threshold test of each step with decisions[i] (a step without a comparable full call

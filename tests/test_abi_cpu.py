@@ -107,3 +107,31 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(8)
     with pytest.raises(moss.MossError):
         moss.cfg_euler_step(x, x, x, 3.0, 1.0, 0.9)
+
+
+def test_sample_options_defaults_and_checks_without_launching():
+    lib = moss.lib()
+    opt = moss.SampleOptions()
+    lib.moss_sample_options_init(ctypes.byref(opt), ctypes.sizeof(moss.SampleOptions))
+    assert opt.struct_size == ctypes.sizeof(moss.SampleOptions)
+    assert opt.cfg_truncation == 1.0 and opt.step_cache_threshold == 0.0
+    assert not opt.cached_out and not opt.change_out
+    before = lib.moss_launch_count(0)
+
+    def call(o):
+        return lib.moss_sample_ex(None, 4, 3.0, 5.0, 42, None, 0, 0.01, 1.0, None, 0, None, 0, 64, 64,
+                                  ctypes.byref(o), None, None)
+
+    bad = moss.SampleOptions()
+    lib.moss_sample_options_init(ctypes.byref(bad), 12)
+    assert call(bad) == 5                                                    # struct_size mismatch
+    for field, value in (("cfg_truncation", 1.5), ("cfg_truncation", -0.1), ("cfg_truncation", float("nan")),
+                         ("step_cache_threshold", -1.0), ("step_cache_threshold", float("nan"))):
+        o = moss.SampleOptions()
+        lib.moss_sample_options_init(ctypes.byref(o), ctypes.sizeof(moss.SampleOptions))
+        setattr(o, field, value)
+        assert call(o) == 1, (field, value)
+    ok = moss.SampleOptions()
+    lib.moss_sample_options_init(ctypes.byref(ok), ctypes.sizeof(moss.SampleOptions))
+    assert call(ok) == 1 and "model" in lib.moss_last_error().decode()   # NULL model
+    assert lib.moss_launch_count(0) == before

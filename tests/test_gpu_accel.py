@@ -1,0 +1,122 @@
+"""GPU parity of the lossy accelerators (moss_sample_ex): CFG truncation and the first-block
+step cache, against the oracle's sample_accelerated (MossInfer integration guide, What works:
+Lossy accelerators; Per-image settings).
+
+The cache decision compares a change measured on BF16-rounded activations with a threshold; the
+oracle measures it in float64.  So the tests replay the GPU's decisions in the oracle and check
+(a) the final latent, (b) the measured changes within a tolerance, (c) that every GPU decision
+agrees with its own measured change, and (d) that it agrees with the oracle's wherever the
+oracle's change is not within 20 % of the threshold.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.moss_oracle as o
+from tests.gpu_common import assert_no_device_error, make_model, psnr
+from synth import TINY, make_text
+
+pytestmark = pytest.mark.gpu
+
+# Change tolerance: the block-0 outputs carry BF16 rounding of the block's update terms (about
+# 2^-9 of terms that are a fraction of the stream), against step-to-step changes of 0.2-3 % of it.
+CHANGE_RTOL = 0.1
+CHANGE_ATOL = 2e-4
+
+
+def _setup(seed=81, n_u=16, steps=8):
+    model, wg, wn = make_model(TINY, seed, max_tokens=32, max_latent_hw=64, max_steps=steps)
+    tc = make_text(1, 16, TINY.hidden, seed + 1)[0]
+    tu = make_text(1, max(n_u, 1), TINY.hidden, seed + 2)[0][:n_u].contiguous()
+    return model, wn, tc, tu
+
+
+def _gpu(model, tc, tu, steps, **kw):
+    args = dict(steps=steps, cfg=3.0, shift=5.0, seed=0, uncond_skip_layers=[1], slg_start=0.01, slg_stop=1.0)
+    args.update(kw)
+    out, cached, change = model.sample_accelerated(tc.cuda(), tu.cuda(), 64, 64, **args)
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), cached, change
+
+
+def _oracle(wn, tc, tu, steps, **kw):
+    args = dict(steps=steps, cfg=3.0, shift=5.0, seed=0, uncond_skip_layers=(1,), slg_start=0.01, slg_stop=1.0)
+    args.update(kw)
+    return o.sample_accelerated(wn, TINY.heads, 64, 64, tc.double().numpy(), tu.double().numpy(), **args)
+
+
+def test_accelerators_off_equal_moss_sample_bitwise():
+    model, wn, tc, tu = _setup(steps=4)
+    a, cached, change = _gpu(model, tc, tu, 4)
+    b = model.sample(tc.cuda(), tu.cuda(), 64, 64, steps=4, cfg=3.0, shift=5.0, seed=0, uncond_skip_layers=[1])
+    assert np.array_equal(a, b.cpu().numpy())
+    assert cached == [False] * 4 and all(math.isnan(c) for c in change)
+    model.close()
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("x", [0.0, 0.5, 0.26, 0.24])
+def test_cfg_truncation_matches_oracle(x):
+    model, wn, tc, tu = _setup(steps=4)
+    out, cached, _ = _gpu(model, tc, tu, 4, cfg_truncation=x)
+    ref, _, _ = _oracle(wn, tc, tu, 4, cfg_truncation=x)
+    assert psnr(ref, out) >= 40.0
+    assert not any(cached)
+    if x == 0.0:  # every step conditional only: the CFG-1 sampler, bitwise
+        b = model.sample(tc.cuda(), tu.cuda(), 64, 64, steps=4, cfg=1.0, shift=5.0, seed=0, uncond_skip_layers=[1])
+        assert np.array_equal(out, b.cpu().numpy())
+    model.close()
+    assert_no_device_error()
+
+
+def _check_cache_run(wn, tc, tu, steps, threshold, out, cached, change, **kw):
+    ref, c_or, ch_or = _oracle(wn, tc, tu, steps, decisions=cached, **kw)
+    assert c_or == cached
+    assert psnr(ref, out) >= 40.0
+    assert cached[0] is False and math.isnan(change[0]) and math.isnan(ch_or[0])
+    for i in range(steps):
+        if math.isnan(ch_or[i]):
+            assert math.isnan(change[i]) and not cached[i]
+            continue
+        assert abs(change[i] - ch_or[i]) <= CHANGE_RTOL * ch_or[i] + CHANGE_ATOL, (i, change[i], ch_or[i])
+        assert cached[i] == (change[i] < threshold)                     # (c) own measurement
+        if abs(ch_or[i] - threshold) > 0.2 * threshold:                  # (d) clear-cut steps
+            assert cached[i] == (ch_or[i] < threshold), (i, ch_or[i], threshold)
+
+
+@pytest.mark.parametrize("threshold", [1e9, 0.008, 0.003])
+def test_step_cache_matches_oracle(threshold):
+    steps = 8
+    model, wn, tc, tu = _setup(steps=steps)
+    out, cached, change = _gpu(model, tc, tu, steps, step_cache_threshold=threshold)
+    if threshold == 1e9:
+        assert cached == [False] + [True] * (steps - 1)
+    assert 0 < sum(cached) < steps if threshold != 1e9 else True
+    _check_cache_run(wn, tc, tu, steps, threshold, out, cached, change, step_cache_threshold=threshold)
+    model.close()
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("n_u", [0, 5])
+def test_step_cache_with_truncation_and_short_negative_prompt(n_u):
+    """Both accelerators on, a negative prompt shorter than the prompt: the switch to one branch
+    forces a full call, and the cache keeps working on the conditional branch after it."""
+    steps = 8
+    model, wn, tc, tu = _setup(seed=91, n_u=n_u, steps=steps)
+    kw = dict(step_cache_threshold=0.01, cfg_truncation=0.5)
+    out, cached, change = _gpu(model, tc, tu, steps, **kw)
+    assert not cached[4] and math.isnan(change[4])                       # first conditional-only step
+    _check_cache_run(wn, tc, tu, steps, 0.01, out, cached, change, **kw)
+    model.close()
+    assert_no_device_error()
+
+
+def test_step_cache_threshold_zero_equals_moss_sample_bitwise():
+    model, wn, tc, tu = _setup(steps=4)
+    a, cached, _ = _gpu(model, tc, tu, 4, step_cache_threshold=0.0)
+    b = model.sample(tc.cuda(), tu.cuda(), 64, 64, steps=4, cfg=3.0, shift=5.0, seed=0, uncond_skip_layers=[1])
+    assert np.array_equal(a, b.cpu().numpy()) and not any(cached)
+    model.close()
+    assert_no_device_error()

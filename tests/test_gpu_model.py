@@ -276,3 +276,28 @@ def test_full_denoise_step_short_negative_prompt(full_model):
     moss.cfg_euler_step(ref, vc[0].contiguous(), vu[0].contiguous(), 3.0, float(sig[3]), float(sig[4]))
     assert rel_l2(x.cpu().numpy(), ref.cpu().numpy()) <= 1e-6
     assert_no_device_error()
+
+
+def test_full_accelerators(full_model):
+    """1024^2, 2 steps of the full model: moss_sample_ex with the accelerators off equals
+    moss_sample; CFG truncation at 0.5 equals a CFG step followed by a conditional-only step;
+    the step cache with a huge threshold reuses the second step with a finite change."""
+    from synth import FULL
+    model, w = full_model
+    tc = make_text(1, 512, FULL.hidden, 31, device="cuda")[0].contiguous()
+    tu = make_text(1, 77, FULL.hidden, 32, device="cuda")[0].contiguous()
+    kw = dict(steps=2, cfg=3.0, shift=5.0, seed=9, uncond_skip_layers=[22], slg_start=0.0, slg_stop=1.0)
+    plain = model.sample(tc, tu, 1024, 1024, **kw).clone()
+    off, cached, change = model.sample_accelerated(tc, tu, 1024, 1024, **kw)
+    assert torch.equal(off, plain) and cached == [False, False]
+    trunc, _, _ = model.sample_accelerated(tc, tu, 1024, 1024, cfg_truncation=0.5, **kw)
+    x = torch.empty(128, 128, 32, device="cuda")
+    moss.init_noise(x, 9)
+    model.denoise_step(x, tc, tu, 1024, 1024, 0, 2, 3.0, 5.0, [22], 0.0, 1.0)
+    model.denoise_step(x, tc, tu, 1024, 1024, 1, 2, 1.0, 5.0, [22], 0.0, 1.0)
+    assert torch.equal(trunc, x)
+    cache, cached, change = model.sample_accelerated(tc, tu, 1024, 1024, step_cache_threshold=1e9, **kw)
+    torch.cuda.synchronize()
+    assert cached == [False, True] and 0.0 < change[1] < 1.0
+    assert torch.isfinite(cache).all() and not torch.equal(cache, plain)
+    assert_no_device_error()
