@@ -49,6 +49,11 @@ Readings taken where the pages are silent (each repeated where it is used):
       o + (x_L - o_ref) of the last full call (blocks 1..L-1 of that call, as a residual).
       Otherwise it runs every block and becomes the last full call.  The first step is
       always a full call.
+  R22 Text projection: a linear layer with bias from the encoder's final-layer states
+      (width 4096) to D.
+  R23 Text-only block: the joint block (R5-R9, R12) on the prompt's tokens alone, positions
+      (j+1, 0, 0), without timestep modulation (shift 0, scale 0, gates 1), so the refined
+      prompt is the same at every step.
 """
 from __future__ import annotations
 
@@ -445,6 +450,34 @@ def sample(w: dict, heads: int, height: int, width: int, text_c: np.ndarray, tex
         v_c = dit_forward(x, np.asarray(text_c)[None], t, [()], w, heads, head_dim)[0].astype(F32)
         v_u = dit_forward(x, np.asarray(text_u)[None], t, [skip_u], w, heads, head_dim)[0].astype(F32)
         x = cfg_euler(x, v_c, v_u, cfg, sig[i], sig[i + 1])
+    return x
+
+
+# --------------------------------------------------------------------------------------
+# Text path.  [WP] Architecture and specs: the frozen text encoder's final-layer states pass
+# through a projection and two text-only blocks before they join the image tokens.
+# Readings R22, R23.
+# --------------------------------------------------------------------------------------
+def text_projection(enc_states: np.ndarray, proj_w: np.ndarray, proj_b: np.ndarray) -> np.ndarray:
+    """R22: [n, enc_dim] -> [n, D]."""
+    return np.asarray(enc_states, F64) @ np.asarray(proj_w, F64).T + np.asarray(proj_b, F64)
+
+
+def unmodulated(D: int) -> np.ndarray:
+    """R23: the modulation vector of a text-only block: shifts and scales 0, gates 1."""
+    m = np.zeros(6 * D, dtype=F64)
+    m[2 * D:3 * D] = 1.0
+    m[5 * D:6 * D] = 1.0
+    return m
+
+
+def text_refine(enc_states: np.ndarray, tw: dict, heads: int, head_dim: int = 128) -> np.ndarray:
+    """The prompt's text states at width D: projection, then each text-only block in order."""
+    x = text_projection(enc_states, tw["proj_w"], tw["proj_b"])
+    angles = rope_angles(token_positions(0, 0, x.shape[0]), head_dim)
+    mod = unmodulated(x.shape[1])
+    for l in range(tw["wqkv"].shape[0]):
+        x = block_forward(x, layer_weights(tw, l), mod, angles, heads, head_dim)
     return x
 
 

@@ -96,6 +96,35 @@ def make_weights(shape: ModelShape, seed: int, device: str = "cpu", layers: int 
     return w
 
 
+TEXT_ENC_DIM = 4096  # width of the text encoder's final-layer states (Qwen3.5-9B)
+TEXT_BLOCKS = 2      # text-only refiner blocks
+
+
+def make_text_weights(shape: ModelShape, seed: int, enc_dim: int = TEXT_ENC_DIM, blocks: int = TEXT_BLOCKS,
+                      device: str = "cpu", std: float = 0.02) -> dict:
+    """Text path parameters: projection [D, enc_dim] + [D] and `blocks` text-only blocks with the
+    joint blocks' linear layers and Q/K gains (stacked like make_weights; no modulation)."""
+    D, F, d = shape.hidden, shape.ffn, shape.head_dim
+    g = make_generator(seed, device)
+    bf = torch.bfloat16
+    w = {}
+    w["proj_w"] = _normal((D, enc_dim), g, device, std, bf)
+    w["proj_b"] = _normal((D,), g, device, std, bf)
+    w["wqkv"] = _normal((blocks, 3 * D, D), g, device, std, bf)
+    w["q_gain"] = 1.0 + _normal((blocks, d), g, device, std)
+    w["k_gain"] = 1.0 + _normal((blocks, d), g, device, std)
+    w["wo"] = _normal((blocks, D, D), g, device, std, bf)
+    w["wg"] = _normal((blocks, F, D), g, device, std, bf)
+    w["wu"] = _normal((blocks, F, D), g, device, std, bf)
+    w["wd"] = _normal((blocks, D, F), g, device, std, bf)
+    return w
+
+
+def make_encoder_states(n_txt: int, seed: int, enc_dim: int = TEXT_ENC_DIM, device: str = "cpu") -> torch.Tensor:
+    """BF16 final-layer text-encoder states [n_txt, enc_dim] ~ N(0, 1) (stand-in for Qwen3.5-9B's)."""
+    return _normal((n_txt, enc_dim), make_generator(seed, device), device, 1.0, torch.bfloat16)
+
+
 def make_latent(h8: int, w8: int, seed: int, channels: int = 32, device: str = "cpu") -> torch.Tensor:
     """FP32 latent [h8, w8, channels] ~ N(0, 1)."""
     return _normal((h8, w8, channels), make_generator(seed, device), device)
