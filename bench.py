@@ -256,6 +256,42 @@ def run_op(args):
     return 0
 
 
+def run_text(args):
+    """The text path once per prompt: projection 4096 -> 3072 and two text-only blocks at full
+    width, for the benchmark's 512-token prompt and the pages' 4096-token maximum.  Prints one JSON
+    line: ms per call (CUDA events) and TFLOP/s of the algorithmic work."""
+    import torch
+
+    import diffusion_transformer_text_block_b200 as moss
+    from synth import ModelShape, make_encoder_states, make_text_weights, make_weights
+
+    shape = ModelShape(layers=1, hidden=3072, heads=24, ffn=8192)
+    D, F = shape.hidden, shape.ffn
+    w = {k: v for k, v in make_weights(shape, 3, device="cuda").items()}
+    model = moss.Model(shape, w, max_tokens=4096, max_batch=1, max_latent_hw=64, max_steps=1)
+    model.set_text_weights(make_text_weights(shape, 4, device="cuda"))
+    out = {"op": "text"}
+    for n in (N_TXT, 4096):
+        enc = make_encoder_states(n, 5, device="cuda")
+        res = torch.empty(n, D, device="cuda")
+        for _ in range(args.warmup):
+            model.text_refine(enc, out=res)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            model.text_refine(enc, out=res)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        flop = 2.0 * n * 4096 * D + 2 * (2.0 * n * D * (4 * D + 3 * F) + 4.0 * n * n * D)
+        out[f"n{n}"] = {"ms": round(ms, 4), "tflops": round(flop / (ms / 1e3) / 1e12, 1)}
+    out["device_status"] = moss.device_status(clear=True)
+    model.close()
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def run_accel(args):
     """Whole 1024^2 images (50 steps, CFG 3, shift 5, uncond skips layer 22 in slg [0.01, 1.0])
     through moss_sample and moss_sample_ex with the lossy accelerators (CFG truncation, the
@@ -312,7 +348,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["block", "attention", "accel"], default=None,
+    ap.add_argument("--op", choices=["block", "attention", "accel", "text"], default=None,
                     help="time one kernel class on the 1024^2 shapes instead of the denoising step; "
                          "'accel' times whole 50-step images with the lossy accelerators")
     args = ap.parse_args()
@@ -320,6 +356,8 @@ def main():
         return run_reference(args)
     if args.op == "accel":
         return run_accel(args)
+    if args.op == "text":
+        return run_text(args)
     if args.op:
         return run_op(args)
 

@@ -43,6 +43,14 @@ class Weights(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32)] + [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
 
 
+TEXT_WEIGHT_FIELDS = ("proj_w", "proj_b", "wqkv", "q_gain", "k_gain", "wo", "wg", "wu", "wd")
+
+
+class TextWeights(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("enc_dim", ctypes.c_int32), ("blocks", ctypes.c_int32)] + \
+        [(n, ctypes.c_void_p) for n in TEXT_WEIGHT_FIELDS]
+
+
 class SampleOptions(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("cfg_truncation", ctypes.c_double),
                 ("step_cache_threshold", ctypes.c_double), ("cached_out", ctypes.POINTER(ctypes.c_int)),
@@ -72,6 +80,9 @@ _SIGS = {
     "moss_init_noise": (_I, [_P, _I64, ctypes.c_uint64, _P]),
     "moss_denoise_step": (_I, [_P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _F, _D, _P, _I, _D, _D, _P]),
     "moss_sample": (_I, [_P, _I, _F, _D, ctypes.c_uint64, _P, _I, _D, _D, _P, _I, _P, _I, _I, _I, _P, _P]),
+    "moss_text_weights_init": (None, [ctypes.POINTER(TextWeights), ctypes.c_uint32]),
+    "moss_text_refiner_set": (_I, [_P, ctypes.POINTER(TextWeights)]),
+    "moss_text_refine": (_I, [_P, _P, _I, _P, _P]),
     "moss_sample_options_init": (None, [ctypes.POINTER(SampleOptions), ctypes.c_uint32]),
     "moss_sample_ex": (_I, [_P, _I, _F, _D, ctypes.c_uint64, _P, _I, _D, _D, _P, _I, _P, _I, _I, _I,
                             ctypes.POINTER(SampleOptions), _P, _P]),
@@ -279,6 +290,33 @@ class Model:
             self.close()
         except Exception:
             pass
+
+    def set_text_weights(self, tw: dict):
+        """Attach the text path: projection [D, enc_dim] + [D] and the text-only blocks' stacked
+        weights (TEXT_WEIGHT_FIELDS; blocks = tw["wqkv"].shape[0], 0 if absent)."""
+        import torch
+        t = TextWeights()
+        lib().moss_text_weights_init(ctypes.byref(t), ctypes.sizeof(TextWeights))
+        t.enc_dim = tw["proj_w"].shape[1]
+        t.blocks = tw["wqkv"].shape[0] if "wqkv" in tw else 0
+        for name in TEXT_WEIGHT_FIELDS:
+            if name not in tw:
+                continue
+            want = torch.float32 if name in ("q_gain", "k_gain") else torch.bfloat16
+            setattr(t, name, _ptr(tw[name], want, name))
+        _check(lib().moss_text_refiner_set(self._h, ctypes.byref(t)))
+        self._text_weights = tw
+        self.enc_dim = t.enc_dim
+
+    def text_refine(self, enc_states, stream=None, out=None):
+        """enc_states: CUDA BF16 [n_txt, enc_dim] -> FP32 [n_txt, D] text states."""
+        import torch
+        n = enc_states.shape[0]
+        if out is None:
+            out = torch.empty(n, self.shape.hidden, device=enc_states.device, dtype=torch.float32)
+        _check(lib().moss_text_refine(self._h, _ptr(enc_states, torch.bfloat16, "enc_states"), n,
+                                      _ptr(out, torch.float32, "out"), _stream(stream)))
+        return out
 
     def block_forward(self, layer: int, x, grid_h: int, grid_w: int, n_txt: int, t: float, stream=None):
         import torch

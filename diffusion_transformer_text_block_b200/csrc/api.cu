@@ -212,6 +212,12 @@ struct moss_model {
   float* cache_res = nullptr;
   double* chg_dev = nullptr;
   double* chg_host = nullptr;  // pinned
+  // text path (moss_text_refiner_set): weights, descriptors, the blocks' fixed modulation
+  bool has_text = false;
+  moss_text_weights tw;
+  std::vector<CUtensorMap> tt_qkv, tt_wo, tt_wg, tt_wu, tt_wd;
+  CUtensorMap tt_proj;
+  float* tt_mod = nullptr;  // [6 D]: shift 0, scale 0, gate 1 (twice)
   // weight descriptors
   std::vector<CUtensorMap> tm_qkv, tm_wo, tm_wg, tm_wu, tm_wd;
   CUtensorMap tm_img, tm_out;
@@ -223,6 +229,34 @@ struct moss_model {
 };
 
 namespace {
+
+// Weight descriptors of `count` stacked blocks ([count, 3D, D] q|k|v, [count, D, D] out,
+// [count, F, D] gate and up, [count, D, F] down), 64 x 128 boxes.
+bool build_block_maps(int D, int F, int count, const void* wqkv_v, const void* wo_v, const void* wg_v,
+                      const void* wu_v, const void* wd_v, std::vector<CUtensorMap>* tqkv, std::vector<CUtensorMap>* two,
+                      std::vector<CUtensorMap>* twg, std::vector<CUtensorMap>* twu, std::vector<CUtensorMap>* twd,
+                      std::string* e) {
+  tqkv->resize(count);
+  two->resize(count);
+  twg->resize(count);
+  twu->resize(count);
+  twd->resize(count);
+  const bf16* wqkv = static_cast<const bf16*>(wqkv_v);
+  const bf16* wo = static_cast<const bf16*>(wo_v);
+  const bf16* wg = static_cast<const bf16*>(wg_v);
+  const bf16* wu = static_cast<const bf16*>(wu_v);
+  const bf16* wd = static_cast<const bf16*>(wd_v);
+  for (int l = 0; l < count; ++l) {
+    const int64_t dd = static_cast<int64_t>(D) * D, df = static_cast<int64_t>(D) * F;
+    if (!make_tmap_bf16_2d(&(*tqkv)[l], wqkv + l * 3 * dd, D, 3 * D, kGemmBoxK, kGemmBoxRows, e) ||
+        !make_tmap_bf16_2d(&(*two)[l], wo + l * dd, D, D, kGemmBoxK, kGemmBoxRows, e) ||
+        !make_tmap_bf16_2d(&(*twg)[l], wg + l * df, D, F, kGemmBoxK, kGemmBoxRows, e) ||
+        !make_tmap_bf16_2d(&(*twu)[l], wu + l * df, D, F, kGemmBoxK, kGemmBoxRows, e) ||
+        !make_tmap_bf16_2d(&(*twd)[l], wd + l * df, F, D, kGemmBoxK, kGemmBoxRows, e))
+      return false;
+  }
+  return true;
+}
 
 int prof_begin(moss_model* m, cudaStream_t s) {
   ++g_launches;
@@ -332,7 +366,19 @@ int compute_modulation(moss_model* m, const float* ts_host, int T, cudaStream_t 
 // rows, [image; text]); mod_l = [6D] of this layer.  Branches of different lengths are
 // supported for two branches (the QKV epilogue maps rows past the first branch onto the
 // second branch's tokens; attention runs per branch).
-int block_impl(moss_model* m, int l, float* x, const std::vector<int>& lens, const float* mod_l, cudaStream_t s) {
+// Tensor maps and Q/K gains of one block's weights (a DiT layer or a text-only block).
+struct LayerRes {
+  const CUtensorMap* qkv;
+  const CUtensorMap* wo;
+  const CUtensorMap* wg;
+  const CUtensorMap* wu;
+  const CUtensorMap* wd;
+  const float* q_gain;
+  const float* k_gain;
+};
+
+int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<int>& lens, const float* mod_l,
+                 cudaStream_t s) {
   const moss_config& c = m->cfg;
   const int D = c.hidden, F = c.ffn, H = c.heads;
   const int nb = static_cast<int>(lens.size());
@@ -353,12 +399,12 @@ int block_impl(moss_model* m, int l, float* x, const std::vector<int>& lens, con
   EpiParams q;
   q.M = M; q.N = 3 * D; q.K = D;
   q.out_bf16 = m->qkv;
-  q.q_gain = m->w.q_gain + static_cast<int64_t>(l) * 128;
-  q.k_gain = m->w.k_gain + static_cast<int64_t>(l) * 128;
+  q.q_gain = lw.q_gain;
+  q.k_gain = lw.k_gain;
   q.rope = m->rope; q.n_tok = lens[0]; q.hidden = D;
   q.split_rows = equal ? 0 : lens[0];
   q.rope_stride = m->rope_n;
-  LAUNCH(m, MOSS_K_GEMM_QKV, s, launch_gemm(kEpiQkv, tm_h, m->tm_qkv[l], m->tm_qkv[l], q, s, m->err), "qkv gemm");
+  LAUNCH(m, MOSS_K_GEMM_QKV, s, launch_gemm(kEpiQkv, tm_h, *lw.qkv, *lw.qkv, q, s, m->err), "qkv gemm");
 
   if (equal) {
     LAUNCH(m, MOSS_K_ATTENTION, s, launch_attention(m->qkv, m->attn, nb, lens[0], H, D, s, m->err, &e),
@@ -376,7 +422,7 @@ int block_impl(moss_model* m, int l, float* x, const std::vector<int>& lens, con
   EpiParams o;
   o.M = M; o.N = D; o.K = D;
   o.out_f32 = x; o.gate = mod_l + 2 * D;
-  LAUNCH(m, MOSS_K_GEMM_OPROJ, s, launch_gemm(kEpiResid, tm_attn, m->tm_wo[l], m->tm_wo[l], o, s, m->err),
+  LAUNCH(m, MOSS_K_GEMM_OPROJ, s, launch_gemm(kEpiResid, tm_attn, *lw.wo, *lw.wo, o, s, m->err),
          "out-projection gemm");
 
   LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(x, mod_l + 3 * D, mod_l + 4 * D, m->h, M, D, 0, 0, 1e-6f, s),
@@ -385,15 +431,21 @@ int block_impl(moss_model* m, int l, float* x, const std::vector<int>& lens, con
   EpiParams g;
   g.M = M; g.N = F; g.K = D;
   g.out_bf16 = m->act;
-  LAUNCH(m, MOSS_K_GEMM_GATEUP, s, launch_gemm(kEpiSwiglu, tm_h, m->tm_wg[l], m->tm_wu[l], g, s, m->err),
+  LAUNCH(m, MOSS_K_GEMM_GATEUP, s, launch_gemm(kEpiSwiglu, tm_h, *lw.wg, *lw.wu, g, s, m->err),
          "gate/up gemm");
 
   EpiParams d;
   d.M = M; d.N = D; d.K = F;
   d.out_f32 = x; d.gate = mod_l + 5 * D;
-  LAUNCH(m, MOSS_K_GEMM_DOWN, s, launch_gemm(kEpiResid, tm_act, m->tm_wd[l], m->tm_wd[l], d, s, m->err),
+  LAUNCH(m, MOSS_K_GEMM_DOWN, s, launch_gemm(kEpiResid, tm_act, *lw.wd, *lw.wd, d, s, m->err),
          "down gemm");
   return MOSS_OK;
+}
+
+int block_impl(moss_model* m, int l, float* x, const std::vector<int>& lens, const float* mod_l, cudaStream_t s) {
+  const LayerRes lw{&m->tm_qkv[l], &m->tm_wo[l], &m->tm_wg[l], &m->tm_wu[l], &m->tm_wd[l],
+                    m->w.q_gain + static_cast<int64_t>(l) * 128, m->w.k_gain + static_cast<int64_t>(l) * 128};
+  return block_impl_w(m, lw, x, lens, mod_l, s);
 }
 
 // The DiT for `batch` branches sharing `latent`, branch b with n_txts[b] text tokens (equal
@@ -728,25 +780,9 @@ int moss_model_create(const moss_config* cfg, const moss_weights* w, moss_model*
   cudaMemset(m->patches, 0, sizeof(bf16) * m->img_cap * 128);
 
   std::string e;
-  m->tm_qkv.resize(L);
-  m->tm_wo.resize(L);
-  m->tm_wg.resize(L);
-  m->tm_wu.resize(L);
-  m->tm_wd.resize(L);
-  const bf16* wqkv = static_cast<const bf16*>(w->wqkv);
-  const bf16* wo = static_cast<const bf16*>(w->wo);
-  const bf16* wg = static_cast<const bf16*>(w->wg);
-  const bf16* wu = static_cast<const bf16*>(w->wu);
-  const bf16* wd = static_cast<const bf16*>(w->wd);
-  for (int l = 0; l < L; ++l) {
-    const int64_t dd = static_cast<int64_t>(D) * D, df = static_cast<int64_t>(D) * F;
-    if (!make_tmap_bf16_2d(&m->tm_qkv[l], wqkv + l * 3 * dd, D, 3 * D, kGemmBoxK, kGemmBoxRows, &e) ||
-        !make_tmap_bf16_2d(&m->tm_wo[l], wo + l * dd, D, D, kGemmBoxK, kGemmBoxRows, &e) ||
-        !make_tmap_bf16_2d(&m->tm_wg[l], wg + l * df, D, F, kGemmBoxK, kGemmBoxRows, &e) ||
-        !make_tmap_bf16_2d(&m->tm_wu[l], wu + l * df, D, F, kGemmBoxK, kGemmBoxRows, &e) ||
-        !make_tmap_bf16_2d(&m->tm_wd[l], wd + l * df, F, D, kGemmBoxK, kGemmBoxRows, &e))
-      return cleanup(MOSS_ERR_CUDA, e);
-  }
+  if (!build_block_maps(D, F, L, w->wqkv, w->wo, w->wg, w->wu, w->wd, &m->tm_qkv, &m->tm_wo, &m->tm_wg, &m->tm_wu,
+                        &m->tm_wd, &e))
+    return cleanup(MOSS_ERR_CUDA, e);
   if (!make_tmap_bf16_2d(&m->tm_img, w->img_w, 128, D, kGemmBoxK, kGemmBoxRows, &e) ||
       !make_tmap_bf16_2d(&m->tm_out, w->out_w, D, 128, kGemmBoxK, kGemmBoxRows, &e))
     return cleanup(MOSS_ERR_CUDA, e);
@@ -760,7 +796,7 @@ void moss_model_free(moss_model* m) {
   if (!m) return;
   cudaDeviceSynchronize();
   void* bufs[] = {m->x,   m->h,  m->qkv,   m->attn,      m->act,      m->patches, m->v,
-                  m->rope, m->mod, m->sc, m->tvals, m->cache_ref, m->cache_res, m->chg_dev};
+                  m->rope, m->mod, m->sc, m->tvals, m->cache_ref, m->cache_res, m->chg_dev, m->tt_mod};
   for (void* p : bufs)
     if (p) cudaFree(p);
   if (m->chg_host) cudaFreeHost(m->chg_host);
@@ -909,6 +945,87 @@ int moss_sample(moss_model* m, int steps, float cfg, double shift, uint64_t seed
     const bool on = slg_on(i, steps, slg_start, slg_stop);
     rc = step_impl(m, latent_out, text_c, n_txt_c, text_u, n_txt_u, height, width, sig[i], sig[i + 1], cfg,
                    on ? uskip : none, m->mod + static_cast<int64_t>(i) * m->mod_stride, s);
+    if (rc) return rc;
+  }
+  return MOSS_OK;
+}
+
+void moss_text_weights_init(moss_text_weights* tw, uint32_t struct_size) {
+  if (!tw || struct_size < sizeof(uint32_t)) return;
+  moss_text_weights d;
+  std::memset(&d, 0, sizeof d);
+  d.enc_dim = 4096;
+  d.blocks = 2;
+  std::memcpy(tw, &d, std::min<size_t>(struct_size, sizeof d));
+  tw->struct_size = struct_size;
+}
+
+int moss_text_refiner_set(moss_model* m, const moss_text_weights* tw) {
+  g_last_error.clear();
+  if (!m || !tw) return fail(MOSS_ERR_INVALID_ARGUMENT, "model and text weights must not be NULL");
+  if (tw->struct_size != sizeof(moss_text_weights))
+    return fail(MOSS_ERR_ABI_MISMATCH, "moss_text_weights.struct_size is not sizeof(moss_text_weights) of this library");
+  if (tw->enc_dim <= 0 || tw->enc_dim % 64)
+    return fail(MOSS_ERR_INVALID_ARGUMENT, "enc_dim must be a positive multiple of 64");
+  if (tw->blocks < 0 || tw->blocks > 8) return fail(MOSS_ERR_INVALID_ARGUMENT, "blocks must lie in 0..8");
+  const void* need[] = {tw->proj_w, tw->proj_b};
+  const void* blk[] = {tw->wqkv, tw->q_gain, tw->k_gain, tw->wo, tw->wg, tw->wu, tw->wd};
+  for (const void* p : need)
+    if (!p || !aligned16(p)) return fail(MOSS_ERR_INVALID_ARGUMENT, "a text weight pointer is NULL or misaligned");
+  if (tw->blocks > 0)
+    for (const void* p : blk)
+      if (!p || !aligned16(p)) return fail(MOSS_ERR_INVALID_ARGUMENT, "a text weight pointer is NULL or misaligned");
+  const int D = m->cfg.hidden, F = m->cfg.ffn;
+  std::string e;
+  m->has_text = false;
+  if (!make_tmap_bf16_2d(&m->tt_proj, tw->proj_w, tw->enc_dim, D, kGemmBoxK, kGemmBoxRows, &e))
+    return fail(MOSS_ERR_CUDA, e);
+  if (tw->blocks > 0 && !build_block_maps(D, F, tw->blocks, tw->wqkv, tw->wo, tw->wg, tw->wu, tw->wd, &m->tt_qkv,
+                                          &m->tt_wo, &m->tt_wg, &m->tt_wu, &m->tt_wd, &e))
+    return fail(MOSS_ERR_CUDA, e);
+  if (!m->tt_mod) {
+    cudaError_t ce = cudaMalloc(&m->tt_mod, sizeof(float) * 6 * D);
+    if (ce != cudaSuccess) {
+      m->tt_mod = nullptr;
+      return fail(MOSS_ERR_OOM, std::string("text modulation vector: ") + cudaGetErrorString(ce));
+    }
+    std::vector<float> mod(6 * static_cast<size_t>(D), 0.f);
+    std::fill(mod.begin() + 2 * D, mod.begin() + 3 * D, 1.f);
+    std::fill(mod.begin() + 5 * D, mod.end(), 1.f);
+    ce = cudaMemcpy(m->tt_mod, mod.data(), sizeof(float) * mod.size(), cudaMemcpyHostToDevice);
+    if (ce != cudaSuccess) return fail(MOSS_ERR_CUDA, std::string("text modulation vector: ") + cudaGetErrorString(ce));
+  }
+  m->tw = *tw;
+  m->has_text = true;
+  return MOSS_OK;
+}
+
+int moss_text_refine(moss_model* m, const void* enc_states, int n_txt, float* text_out, void* stream) {
+  g_last_error.clear();
+  if (!m || !m->has_text) return fail(MOSS_ERR_INVALID_ARGUMENT, "no text path attached to the model");
+  if (!enc_states || !text_out || !aligned16(enc_states) || !aligned16(text_out))
+    return fail(MOSS_ERR_INVALID_ARGUMENT, "enc_states and text_out must be non-NULL and 16-byte aligned");
+  if (n_txt < 1 || n_txt > m->cfg.max_tokens)
+    return fail(MOSS_ERR_INVALID_ARGUMENT, "n_txt must lie in 1..max_tokens");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = m->cfg.hidden;
+  std::string e;
+  CUtensorMap tm_e;
+  if (!make_tmap_bf16_2d(&tm_e, enc_states, m->tw.enc_dim, n_txt, kGemmBoxK, kGemmBoxRows, &e))
+    return fail(MOSS_ERR_CUDA, e);
+  EpiParams pe;
+  pe.M = n_txt; pe.N = D; pe.K = m->tw.enc_dim;
+  pe.out_f32 = text_out; pe.bias = static_cast<const bf16*>(m->tw.proj_b);
+  pe.n_tok = n_txt; pe.n_branch = 1;
+  LAUNCH(m, MOSS_K_OTHER, s, launch_gemm(kEpiEmbed, tm_e, m->tt_proj, m->tt_proj, pe, s, m->err), "text projection");
+  if (m->tw.blocks == 0) return MOSS_OK;
+  int rc = ensure_rope(m, 0, 0, n_txt, s);
+  if (rc) return rc;
+  const std::vector<int> lens(1, n_txt);
+  for (int b = 0; b < m->tw.blocks; ++b) {
+    const LayerRes lw{&m->tt_qkv[b], &m->tt_wo[b], &m->tt_wg[b], &m->tt_wu[b], &m->tt_wd[b],
+                      m->tw.q_gain + static_cast<int64_t>(b) * 128, m->tw.k_gain + static_cast<int64_t>(b) * 128};
+    rc = block_impl_w(m, lw, text_out, lens, m->tt_mod, s);
     if (rc) return rc;
   }
   return MOSS_OK;

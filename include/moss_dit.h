@@ -214,6 +214,49 @@ int moss_sample(moss_model* m, int steps, float cfg, double shift, uint64_t seed
                 const float* text_c, int n_txt_c, const float* text_u, int n_txt_u, int height, int width,
                 float* latent_out, void* stream);
 
+/* ------------------------------------------------------------------------------------ */
+/* Text path ([WP] Architecture and specs: the frozen text encoder's final-layer states   */
+/* pass through a projection and two text-only blocks).                                 */
+/* ------------------------------------------------------------------------------------ */
+/* Device pointers to the text-path parameters (BF16 except the FP32 gains, 16-byte aligned,
+ * caller-owned, kept alive and unchanged while attached to a model). */
+typedef struct moss_text_weights {
+  uint32_t struct_size;  /* sizeof(moss_text_weights) as compiled by the caller              */
+  int32_t enc_dim;       /* width of the encoder's final-layer states: 4096; multiple of 64   */
+  int32_t blocks;        /* text-only blocks: 2; 0..8 (0 = projection only)                   */
+  const void* proj_w;    /* [D, enc_dim]  projection                                          */
+  const void* proj_b;    /* [D]                                                               */
+  const void* wqkv;      /* [blocks, 3D, D] the joint blocks' layouts, one per text-only block */
+  const float* q_gain;   /* [blocks, 128]                                                     */
+  const float* k_gain;   /* [blocks, 128]                                                     */
+  const void* wo;        /* [blocks, D, D]                                                    */
+  const void* wg;        /* [blocks, F, D]                                                    */
+  const void* wu;        /* [blocks, F, D]                                                    */
+  const void* wd;        /* [blocks, D, F]                                                    */
+} moss_text_weights;
+
+/* Zero pointers, enc_dim 4096, blocks 2; struct_size as given. */
+void moss_text_weights_init(moss_text_weights* tw, uint32_t struct_size);
+
+/* Attach the text path to a model (replacing any attached before).  Builds the weight
+ * descriptors and a 6*D-float device vector for the blocks' fixed modulation.  Synchronous.
+ * Errors: MOSS_ERR_ABI_MISMATCH (struct_size), MOSS_ERR_INVALID_ARGUMENT (NULL model, enc_dim
+ * not a positive multiple of 64, blocks outside 0..8, a NULL or misaligned pointer),
+ * MOSS_ERR_OOM. */
+int moss_text_refiner_set(moss_model* m, const moss_text_weights* tw);
+
+/* The prompt's text states at width D from the encoder's final-layer states: text = enc W_p^T +
+ * b_p, then each text-only block in order: the joint block on the prompt's tokens alone
+ * (positions (j+1, 0, 0)) without timestep modulation (shifts and scales 0, gates 1), so the
+ * result serves every step of a sampling run (readings of the pages' one-line description).
+ *   enc_states: device BF16 [n_txt, enc_dim];  text_out: device FP32 [n_txt, D] (also the
+ *   blocks' residual stream).  1 <= n_txt <= max_tokens.
+ * Uses the model's workspace (calls on one model must not overlap) and replaces its cached
+ * RoPE table, which the next image call rebuilds.
+ * Errors: MOSS_ERR_INVALID_ARGUMENT (no text path attached, NULL or misaligned buffers, n_txt out
+ * of range). */
+int moss_text_refine(moss_model* m, const void* enc_states, int n_txt, float* text_out, void* stream);
+
 /* Lossy accelerators of the sampling loop, both off by default ([MI] What works: Lossy
  * accelerators; Per-image settings: CFG truncation, Step cache).  They change the image. */
 typedef struct moss_sample_options {

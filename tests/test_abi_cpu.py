@@ -135,3 +135,16 @@ def test_sample_options_defaults_and_checks_without_launching():
     lib.moss_sample_options_init(ctypes.byref(ok), ctypes.sizeof(moss.SampleOptions))
     assert call(ok) == 1 and "model" in lib.moss_last_error().decode()   # NULL model
     assert lib.moss_launch_count(0) == before
+
+
+def test_text_path_entry_points_check_arguments_without_launching():
+    lib = moss.lib()
+    tw = moss.TextWeights()
+    lib.moss_text_weights_init(ctypes.byref(tw), ctypes.sizeof(moss.TextWeights))
+    assert tw.struct_size == ctypes.sizeof(moss.TextWeights) and tw.enc_dim == 4096 and tw.blocks == 2
+    assert not tw.proj_w and not tw.wqkv
+    before = lib.moss_launch_count(0)
+    assert lib.moss_text_refiner_set(None, ctypes.byref(tw)) == 1
+    assert lib.moss_text_refine(None, ctypes.c_void_p(16), 4, ctypes.c_void_p(16), None) == 1
+    assert "no text path" in lib.moss_last_error().decode()
+    assert lib.moss_launch_count(0) == before
