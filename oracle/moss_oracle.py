@@ -54,6 +54,10 @@ Readings taken where the pages are silent (each repeated where it is used):
   R23 Text-only block: the joint block (R5-R9, R12) on the prompt's tokens alone, positions
       (j+1, 0, 0), without timestep modulation (shift 0, scale 0, gates 1), so the refined
       prompt is the same at every step.
+  R24 Three-pass SLG (slg_scale > 0; parity unpinned: the pages give no formula): inside the
+      skip window a third pass runs the conditional branch with the skip layers left out
+      (v_cs), and v = v_u + cfg (v_c - v_u) + slg_scale (v_c - v_cs) in FP32; outside the
+      window, and on CFG-truncated steps, the two-pass rule holds.
 """
 from __future__ import annotations
 
@@ -134,6 +138,13 @@ def euler_update(x: np.ndarray, v: np.ndarray, sigma: float, sigma_next: float) 
 def cfg_euler(x, v_c, v_u, cfg, sigma, sigma_next):
     """One guided Euler step: x + (sigma' - sigma) * (v_u + cfg (v_c - v_u))."""
     return euler_update(x, cfg_combine(v_c, v_u, cfg), sigma, sigma_next)
+
+
+def slg_combine(v_c: np.ndarray, v_u: np.ndarray, v_cs: np.ndarray, cfg: float, slg_scale: float) -> np.ndarray:
+    """R24 (parity unpinned): the CFG combine plus slg_scale (v_c - v_cs), in FP32."""
+    v_c = np.asarray(v_c, F32)
+    v_cs = np.asarray(v_cs, F32)
+    return (cfg_combine(v_c, v_u, cfg) + F32(slg_scale) * (v_c - v_cs)).astype(F32)
 
 
 # --------------------------------------------------------------------------------------
@@ -504,8 +515,10 @@ def sample_accelerated(w: dict, heads: int, height: int, width: int, text_c: np.
                        steps: int = 50, cfg: float = 3.0, shift: float = 5.0, seed: int = 42,
                        uncond_skip_layers=(22,), slg_start: float = 0.01, slg_stop: float = 1.0,
                        cfg_truncation: float = 1.0, step_cache_threshold: float = 0.0, decisions=None,
-                       head_dim: int = 128, x0: np.ndarray | None = None):
-    """The sampler of `sample` with CFG truncation (R19) and the step cache (R20, R21).
+                       slg_scale: float = 0.0, head_dim: int = 128, x0: np.ndarray | None = None):
+    """The sampler of `sample` with CFG truncation (R19), the step cache (R20, R21) and
+    three-pass SLG (R24; slg_scale 0 keeps the two-pass recipe).  Branch order of a call:
+    conditional, skipped conditional (three-pass steps only), unconditional.
 
     step_cache_threshold <= 0 turns the cache off.  `decisions`, when given, replaces the
     threshold test of each step with decisions[i] (a step without a comparable full call
@@ -529,9 +542,16 @@ def sample_accelerated(w: dict, heads: int, height: int, width: int, text_c: np.
     for i in range(steps):
         t = float(sig[i])
         two = cfg != 1.0 and not cfg_truncated(i, steps, cfg_truncation)
-        texts = [np.asarray(text_c, F64), np.asarray(text_u, F64)] if two else [np.asarray(text_c, F64)]
-        skip_u = tuple(uncond_skip_layers) if slg_active(i, steps, slg_start, slg_stop) else ()
-        skips = [(), skip_u] if two else [()]
+        window = slg_active(i, steps, slg_start, slg_stop)
+        three = two and slg_scale > 0.0 and window
+        skip_u = tuple(uncond_skip_layers) if window else ()
+        tc, tu = np.asarray(text_c, F64), np.asarray(text_u, F64)
+        if three:
+            texts, skips = [tc, tc, tu], [(), skip_u, skip_u]
+        elif two:
+            texts, skips = [tc, tu], [(), skip_u]
+        else:
+            texts, skips = [tc], [()]
         c = conditioning(t, w)
         mods = [block_modulation(c, w["mod_w"][l], w["mod_b"][l]) for l in range(L)]
         img = patchify(np.asarray(x, F64)) @ w["img_w"].T + w["img_b"]
@@ -560,7 +580,9 @@ def sample_accelerated(w: dict, heads: int, height: int, width: int, text_c: np.
             if use_cache:
                 last = (len(texts), o0, [xl[b] - o0[b] for b in range(len(texts))])
         v = [unpatchify(final_layer(xb[:n_img], c, w), h8, w8, 32).astype(F32) for xb in xl]
-        if two:
+        if three:
+            x = euler_update(x, slg_combine(v[0], v[2], v[1], cfg, slg_scale), sig[i], sig[i + 1])
+        elif two:
             x = cfg_euler(x, v[0], v[1], cfg, sig[i], sig[i + 1])
         else:
             x = euler_update(x, v[0], sig[i], sig[i + 1])

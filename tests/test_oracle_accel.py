@@ -148,3 +148,59 @@ def test_step_cache_full_call_after_branch_count_changes():
     _, cached, change = _run(w, tc, tu, x0, step_cache_threshold=1e-9, cfg_truncation=0.5)
     assert cached == [False, True, False, True]
     assert math.isnan(change[2])
+
+
+# Three-pass SLG (reading R24; the pages name the option and the extra skipped conditional
+# pass but give no formula, so these pins check the reading's arithmetic and its invariants,
+# not the pages).
+def test_slg_combine_closed_forms():
+    rng = np.random.default_rng(3)
+    vc, vu, vcs = (rng.standard_normal(64).astype(np.float32) for _ in range(3))
+    np.testing.assert_array_equal(o.slg_combine(vc, vu, vcs, 3.0, 0.0), o.cfg_combine(vc, vu, 3.0))
+    np.testing.assert_array_equal(o.slg_combine(vc, vu, vc, 3.0, 2.5), o.cfg_combine(vc, vu, 3.0))
+    np.testing.assert_allclose(o.slg_combine(vc, vu, vcs, 1.0, 2.0), vc + 2.0 * (vc - vcs), rtol=1e-6, atol=1e-6)
+
+
+def test_three_pass_off_and_outside_window_are_two_pass():
+    w, tc, tu, x0 = _setup()
+    ref, _, _ = _run(w, tc, tu, x0)
+    a, _, _ = _run(w, tc, tu, x0, slg_scale=0.0)
+    b, _, _ = _run(w, tc, tu, x0, slg_scale=2.0, slg_start=2.0, slg_stop=3.0)  # window never active
+    np.testing.assert_array_equal(a, ref)
+    # outside the window the uncond branch does not skip either: compare with a two-pass run
+    # that has the same (inactive) window
+    ref2, _, _ = _run(w, tc, tu, x0, slg_start=2.0, slg_stop=3.0)
+    np.testing.assert_array_equal(b, ref2)
+
+
+def test_three_pass_is_cfg_plus_scaled_skip_difference():
+    """Inside the window: v = CFG(v_c, v_u) + s (v_c - v_cs) with v_cs the conditional forward
+    skipping the SLG layers, composed here from the pinned single-branch forward."""
+    w, tc, tu, x0 = _setup()
+    out, _, _ = _run(w, tc, tu, x0, slg_scale=2.0, steps=2)
+    sig = o.sigma_schedule(2, 5.0)
+    x = x0
+    for i in range(2):
+        su = (1,) if o.slg_active(i, 2, 0.01, 1.0) else ()
+        vc = o.dit_forward(x, tc[None], float(sig[i]), [()], w, TINY.heads)[0].astype(np.float32)
+        vu = o.dit_forward(x, tu[None], float(sig[i]), [su], w, TINY.heads)[0].astype(np.float32)
+        if su:
+            vcs = o.dit_forward(x, tc[None], float(sig[i]), [su], w, TINY.heads)[0].astype(np.float32)
+            v = o.slg_combine(vc, vu, vcs, 3.0, 2.0)
+        else:
+            v = o.cfg_combine(vc, vu, 3.0)
+        x = o.euler_update(x, v, sig[i], sig[i + 1])
+    np.testing.assert_array_equal(out, x)
+
+
+def test_three_pass_with_identity_skip_layer_is_two_pass():
+    """When the skipped layer adds nothing (its gates are zero), v_cs = v_c and the third pass
+    changes nothing."""
+    w, tc, tu, x0 = _setup()
+    D = TINY.hidden
+    w["mod_w"][1] = 0.0
+    w["mod_b"][1][2 * D:3 * D] = 0.0
+    w["mod_b"][1][5 * D:6 * D] = 0.0
+    a, _, _ = _run(w, tc, tu, x0, slg_scale=2.0)
+    b, _, _ = _run(w, tc, tu, x0)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-6)
