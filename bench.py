@@ -256,6 +256,67 @@ def run_op(args):
     return 0
 
 
+def run_c5(args):
+    """The long-sequence stress workload: 2048^2 (16384 image tokens) with a 4096-token prompt
+    (20480 tokens per branch), full 42-block DiT, CFG batch 2, skip layer 22, 10 Euler steps at
+    shift 5.  Times --steps of those steps (default all 10) after --warmup, with per-class device
+    time; prints one JSON line."""
+    import torch
+
+    import diffusion_transformer_text_block_b200 as moss
+    from synth import FULL, make_text, make_weights
+
+    H = W = 2048
+    n_txt, n_steps = 4096, 10
+    N = (H // 16) * (W // 16) + n_txt
+    w = make_weights(FULL, 2, device="cuda")
+    model = moss.Model(FULL, w, max_tokens=N, max_batch=2, max_latent_hw=(H // 8) * (W // 8), max_steps=1)
+    tc = make_text(1, n_txt, FULL.hidden, 100, device="cuda")[0].contiguous()
+    tu = make_text(1, n_txt, FULL.hidden, 200, device="cuda")[0].contiguous()
+    x = torch.empty(H // 8, W // 8, 32, device="cuda")
+    moss.init_noise(x, 42)
+    steps = min(args.steps, n_steps)
+
+    def step(i):
+        model.denoise_step(x, tc, tu, H, W, i, n_steps, CFG, SHIFT, SKIP, *SLG)
+
+    for i in range(min(args.warmup, 1)):
+        step(i)
+    torch.cuda.synchronize()
+    model.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    prof = model.profile_read()
+    peaks = read_peaks()
+    bl = sum(2 * FULL.layers - (len(SKIP) if _slg_on(i, n_steps, *SLG) else 0) for i in range(steps))
+    fl = flops_per_branch_layer(N)
+    out = {"op": "c5", "workload": "2048^2, 16384 image + 4096 text tokens per branch, CFG batch 2, skip layer 22, "
+           "10 Euler steps, shift 5, random-init 42-block DiT", "s_per_step": round(ms / 1e3, 4),
+           "s_per_10_steps": round(ms * n_steps / 1e3, 3), "steps_timed": steps, "kernels": {}}
+    total = 0.0
+    for k, (n, tms) in prof.items():
+        if not n:
+            continue
+        rec = {"launches": n, "ms": round(tms, 3)}
+        total += tms
+        if k in fl:
+            tf = bl * fl[k] / (tms / 1e3) / 1e12
+            rec["tflops"] = round(tf, 1)
+            rec["frac"] = round(tf / peaks["bf16_tflops_sustained"], 4)
+        out["kernels"][k] = rec
+    for k in out["kernels"]:
+        out["kernels"][k]["share"] = round(out["kernels"][k]["ms"] / total, 4)
+    out["device_status"] = moss.device_status(clear=True)
+    model.close()
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def run_text(args):
     """The text path once per prompt: projection 4096 -> 3072 and two text-only blocks at full
     width, for the benchmark's 512-token prompt and the pages' 4096-token maximum.  Prints one JSON
@@ -295,7 +356,8 @@ def run_text(args):
 def run_accel(args):
     """Whole 1024^2 images (50 steps, CFG 3, shift 5, uncond skips layer 22 in slg [0.01, 1.0])
     through moss_sample and moss_sample_ex with the lossy accelerators (CFG truncation, the
-    first-block step cache at the pages' default thresholds 0.02 and 0.03).  Random-init
+    first-block step cache at the pages' default thresholds 0.02 and 0.03) and with three-pass
+    skip-layer guidance (a third branch inside the window).  Random-init
     weights: how often the cache engages depends on the weights, so the reuse counts here say
     nothing about a trained model.  Prints one JSON line: seconds per image (CUDA events around
     each call) and the number of reused steps."""
@@ -305,14 +367,15 @@ def run_accel(args):
     from synth import FULL, make_text, make_weights
 
     w = make_weights(FULL, 2, device="cuda")
-    model = moss.Model(FULL, w, max_tokens=4096 + N_TXT, max_batch=2, max_latent_hw=128 * 128, max_steps=50)
+    model = moss.Model(FULL, w, max_tokens=4096 + N_TXT, max_batch=3, max_latent_hw=128 * 128, max_steps=50)
     tc = make_text(1, N_TXT, FULL.hidden, 100, device="cuda")[0].contiguous()
     tu = make_text(1, N_TXT, FULL.hidden, 200, device="cuda")[0].contiguous()
     kw = dict(steps=STEPS_PER_IMAGE, cfg=CFG, shift=SHIFT, seed=42, uncond_skip_layers=SKIP, slg_start=SLG[0],
               slg_stop=SLG[1])
     runs = [("plain", None), ("cfg_truncation_0.5", dict(cfg_truncation=0.5)),
             ("step_cache_0.02", dict(step_cache_threshold=0.02)), ("step_cache_0.03", dict(step_cache_threshold=0.03)),
-            ("both_0.5_0.03", dict(cfg_truncation=0.5, step_cache_threshold=0.03))]
+            ("both_0.5_0.03", dict(cfg_truncation=0.5, step_cache_threshold=0.03)),
+            ("three_pass_slg_2.0", dict(slg_scale=2.0))]
     model.sample(tc, tu, HEIGHT, WIDTH, **dict(kw, steps=2))  # warm-up
     torch.cuda.synchronize()
     out = {"op": "accel", "workload": "1024^2 image, 50 steps, CFG 3, random-init 42-block DiT", "runs": {}}
@@ -348,7 +411,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["block", "attention", "accel", "text"], default=None,
+    ap.add_argument("--op", choices=["block", "attention", "accel", "text", "c5"], default=None,
                     help="time one kernel class on the 1024^2 shapes instead of the denoising step; "
                          "'accel' times whole 50-step images with the lossy accelerators")
     args = ap.parse_args()
@@ -358,6 +421,8 @@ def main():
         return run_accel(args)
     if args.op == "text":
         return run_text(args)
+    if args.op == "c5":
+        return run_c5(args)
     if args.op:
         return run_op(args)
 

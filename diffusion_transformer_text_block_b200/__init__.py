@@ -53,7 +53,8 @@ class TextWeights(ctypes.Structure):
 
 class SampleOptions(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("cfg_truncation", ctypes.c_double),
-                ("step_cache_threshold", ctypes.c_double), ("cached_out", ctypes.POINTER(ctypes.c_int)),
+                ("step_cache_threshold", ctypes.c_double), ("slg_scale", ctypes.c_double),
+                ("cached_out", ctypes.POINTER(ctypes.c_int)),
                 ("change_out", ctypes.POINTER(ctypes.c_float))]
 
 
@@ -368,7 +369,7 @@ class Model:
     def sample_accelerated(self, text_c, text_u, height: int, width: int, steps: int = 50, cfg: float = 3.0,
                            shift: float = 5.0, seed: int = 42, uncond_skip_layers: Sequence[int] = (22,),
                            slg_start: float = 0.01, slg_stop: float = 1.0, cfg_truncation: float = 1.0,
-                           step_cache_threshold: float = 0.0, stream=None, out=None):
+                           step_cache_threshold: float = 0.0, slg_scale: float = 0.0, stream=None, out=None):
         """moss_sample_ex: returns (latent, cached [steps] list of bool, change [steps] list of float)."""
         import torch
         if out is None:
@@ -380,6 +381,7 @@ class Model:
         lib().moss_sample_options_init(ctypes.byref(opt), ctypes.sizeof(SampleOptions))
         opt.cfg_truncation = cfg_truncation
         opt.step_cache_threshold = step_cache_threshold
+        opt.slg_scale = slg_scale
         cached = (ctypes.c_int * steps)()
         change = (ctypes.c_float * steps)()
         opt.cached_out = ctypes.cast(cached, ctypes.POINTER(ctypes.c_int))

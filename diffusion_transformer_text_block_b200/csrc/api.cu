@@ -402,7 +402,9 @@ int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<
   q.q_gain = lw.q_gain;
   q.k_gain = lw.k_gain;
   q.rope = m->rope; q.n_tok = lens[0]; q.hidden = D;
-  q.split_rows = equal ? 0 : lens[0];
+  // Branches of unequal lengths: every branch but the last has lens[0] tokens (the callers
+  // order them so), the last one starts at split_rows.
+  q.split_rows = equal ? 0 : static_cast<int>(M - lens[nb - 1]);
   q.rope_stride = m->rope_n;
   LAUNCH(m, MOSS_K_GEMM_QKV, s, launch_gemm(kEpiQkv, tm_h, *lw.qkv, *lw.qkv, q, s, m->err), "qkv gemm");
 
@@ -470,15 +472,14 @@ int embed_impl(moss_model* m, int batch, const float* latent, const float* const
   r.lens.assign(batch, 0);
   r.off.assign(batch + 1, 0);
   int n_txt_max = 0;
-  bool equal = true;
   for (int b = 0; b < batch; ++b) {
     r.lens[b] = r.n_img + n_txts[b];
     r.off[b + 1] = r.off[b] + r.lens[b];
     n_txt_max = std::max(n_txt_max, n_txts[b]);
-    equal = equal && n_txts[b] == n_txts[0];
   }
-  if (!equal && batch > 2)
-    return fail(MOSS_ERR_UNSUPPORTED, "branches of different text lengths are supported for two branches");
+  for (int b = 1; b + 1 < batch; ++b)
+    if (n_txts[b] != n_txts[0])
+      return fail(MOSS_ERR_UNSUPPORTED, "only the last branch may have a text length different from the first's");
   int rc = ensure_rope(m, r.gh, r.gw, n_txt_max, s);
   if (rc) return rc;
 
@@ -527,7 +528,7 @@ int final_impl(moss_model* m, const CallRows& r, const float* mod, float* v_out,
   const int D = m->cfg.hidden, L = m->cfg.layers;
   const float* fmod = mod + static_cast<int64_t>(L) * 6 * D;
   const int rows = r.batch * r.n_img;
-  // Image rows of branch b start at b * lens[0] (equal lengths, or two branches).
+  // Image rows of branch b start at b * lens[0] (every branch but the last has lens[0] rows).
   LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(m->x, fmod, fmod + D, m->h, rows, D, r.n_img, r.lens[0], 1e-6f, s),
          "final ln");
   std::string e;
@@ -611,15 +612,23 @@ int ensure_cache_buffers(moss_model* m) {
 // One step of the sampling loop with the lossy accelerators: `two` = run the unconditional
 // branch (false once CFG truncation has dropped it); threshold > 0 = first-block step cache.
 int accel_step_impl(moss_model* m, float* x, const float* text_c, int n_txt_c, const float* text_u, int n_txt_u,
-                    int height, int width, float sigma, float sigma_next, float cfg, bool two,
+                    int height, int width, float sigma, float sigma_next, float cfg, bool two, float slg_scale,
                     const std::vector<char>& uskip, const float* mod, double threshold, StepCache* sc, int* cached,
                     float* change, cudaStream_t s) {
-  const int batch = two ? 2 : 1;
+  // Branches: conditional, then (three-pass SLG) the conditional with the skip layers left
+  // out, then the unconditional; every branch but the last has the prompt's length.
+  const bool three = two && slg_scale > 0.0f;
+  const int batch = three ? 3 : (two ? 2 : 1);
   const int D = m->cfg.hidden, L = m->cfg.layers;
   std::vector<std::vector<char>> skips(batch, std::vector<char>(L, 0));
-  if (two) skips[1] = uskip;
-  const float* texts[2] = {text_c, text_u};
-  const int n_txts[2] = {n_txt_c, n_txt_u};
+  const float* texts[3] = {text_c, text_u, text_u};
+  int n_txts[3] = {n_txt_c, n_txt_u, n_txt_u};
+  if (two) skips[batch - 1] = uskip;
+  if (three) {
+    skips[1] = uskip;
+    texts[1] = text_c;
+    n_txts[1] = n_txt_c;
+  }
   CallRows r;
   int rc = embed_impl(m, batch, x, texts, n_txts, height, width, &r, s);
   if (!rc) rc = blocks_impl(m, 0, 1, r, mod, skips, s);
@@ -659,9 +668,15 @@ int accel_step_impl(moss_model* m, float* x, const float* text_c, int n_txt_c, c
   rc = final_impl(m, r, mod, m->v, s);
   if (rc) return rc;
   const int64_t nl = static_cast<int64_t>(height / 8) * (width / 8) * 32;
-  const float* vu = two ? m->v + nl : m->v;
-  LAUNCH(m, MOSS_K_CFG_EULER, s, launch_cfg_euler(x, m->v, vu, nl, two ? cfg : 1.0f, sigma, sigma_next, s),
-         "cfg euler");
+  if (three) {
+    LAUNCH(m, MOSS_K_CFG_EULER, s,
+           launch_cfg_slg_euler(x, m->v, m->v + nl, m->v + 2 * nl, nl, cfg, slg_scale, sigma, sigma_next, s),
+           "cfg slg euler");
+  } else {
+    const float* vu = two ? m->v + nl : m->v;
+    LAUNCH(m, MOSS_K_CFG_EULER, s, launch_cfg_euler(x, m->v, vu, nl, two ? cfg : 1.0f, sigma, sigma_next, s),
+           "cfg euler");
+  }
   *cached = reuse ? 1 : 0;
   *change = static_cast<float>(ch);
   return MOSS_OK;
@@ -1037,6 +1052,7 @@ void moss_sample_options_init(moss_sample_options* opt, uint32_t struct_size) {
   std::memset(&d, 0, sizeof d);
   d.cfg_truncation = 1.0;
   d.step_cache_threshold = 0.0;
+  d.slg_scale = 0.0;
   std::memcpy(opt, &d, std::min<size_t>(struct_size, sizeof d));
   opt->struct_size = struct_size;
 }
@@ -1058,6 +1074,8 @@ int moss_sample_ex(moss_model* m, int steps, float cfg, double shift, uint64_t s
     return fail(MOSS_ERR_INVALID_ARGUMENT, "cfg_truncation must lie in [0, 1]");
   if (!(opt.step_cache_threshold >= 0.0))
     return fail(MOSS_ERR_INVALID_ARGUMENT, "step_cache_threshold must be >= 0");
+  if (!(opt.slg_scale >= 0.0 && opt.slg_scale < 1e30))
+    return fail(MOSS_ERR_INVALID_ARGUMENT, "slg_scale must be finite and >= 0");
   if (!m) return fail(MOSS_ERR_INVALID_ARGUMENT, "model is NULL");
   if (steps < 1 || steps > m->cfg.max_steps || !(shift > 0.0))
     return fail(MOSS_ERR_INVALID_ARGUMENT, "need 1 <= steps <= max_steps and shift > 0");
@@ -1065,6 +1083,10 @@ int moss_sample_ex(moss_model* m, int steps, float cfg, double shift, uint64_t s
   int rc = check_step_args(m, latent_out, text_c, n_txt_c, text_u, n_txt_u, height, width, cfg, uncond_skip_layers,
                            n_skip, &uskip);
   if (rc) return rc;
+  if (opt.slg_scale > 0.0 && cfg != 1.0f) {
+    rc = check_tokens(m, 3, height / 16, width / 16, std::max(n_txt_c, n_txt_u));
+    if (rc) return rc;
+  }
   const double thr = opt.step_cache_threshold;
   if (thr > 0.0) {
     rc = ensure_cache_buffers(m);
@@ -1085,7 +1107,7 @@ int moss_sample_ex(moss_model* m, int steps, float cfg, double shift, uint64_t s
     int cached = 0;
     float change = 0.f;
     rc = accel_step_impl(m, latent_out, text_c, n_txt_c, text_u, n_txt_u, height, width, sig[i], sig[i + 1], cfg,
-                         two, on ? uskip : none, m->mod + static_cast<int64_t>(i) * m->mod_stride, thr, &sc,
+                         two, on ? static_cast<float>(opt.slg_scale) : 0.0f, on ? uskip : none, m->mod + static_cast<int64_t>(i) * m->mod_stride, thr, &sc,
                          &cached, &change, s);
     if (rc) return rc;
     if (opt.cached_out) opt.cached_out[i] = cached;

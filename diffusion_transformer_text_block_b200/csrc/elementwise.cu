@@ -110,6 +110,32 @@ __global__ void __launch_bounds__(256) cfg_euler_kernel(float* __restrict__ x, c
   }
 }
 
+// Three-pass skip-layer guidance: the CFG combine plus slg (vc - vcs), then the Euler update.
+__global__ void __launch_bounds__(256) cfg_slg_euler_kernel(float* __restrict__ x, const float* __restrict__ vc,
+                                                            const float* __restrict__ vcs,
+                                                            const float* __restrict__ vu, int64_t n, float cfg,
+                                                            float slg, float dt) {
+  const int64_t n4 = n >> 2;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  float4* x4 = reinterpret_cast<float4*>(x);
+  const float4* c4 = reinterpret_cast<const float4*>(vc);
+  const float4* s4 = reinterpret_cast<const float4*>(vcs);
+  const float4* u4 = reinterpret_cast<const float4*>(vu);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    float4 a = x4[i];
+    const float4 c = __ldcs(c4 + i), k = __ldcs(s4 + i), u = __ldcs(u4 + i);
+    a.x = fmaf(dt, fmaf(slg, c.x - k.x, fmaf(cfg, c.x - u.x, u.x)), a.x);
+    a.y = fmaf(dt, fmaf(slg, c.y - k.y, fmaf(cfg, c.y - u.y, u.y)), a.y);
+    a.z = fmaf(dt, fmaf(slg, c.z - k.z, fmaf(cfg, c.z - u.z, u.z)), a.z);
+    a.w = fmaf(dt, fmaf(slg, c.w - k.w, fmaf(cfg, c.w - u.w, u.w)), a.w);
+    x4[i] = a;
+  }
+  if (blockIdx.x == 0 && threadIdx.x < (n & 3)) {
+    const int64_t i = (n4 << 2) + threadIdx.x;
+    x[i] = fmaf(dt, fmaf(slg, vc[i] - vcs[i], fmaf(cfg, vc[i] - vu[i], vu[i])), x[i]);
+  }
+}
+
 // ---------------------------------------------------------------------------- noise
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): counter (g_lo, g_hi, 0, 0) for the
 // group g of four outputs, key (seed_lo, seed_hi); Box-Muller on ((b >> 9) + 1/2) / 2^23.
@@ -317,6 +343,18 @@ cudaError_t launch_cfg_euler(float* x, const float* vc, const float* vu, int64_t
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
   cfg_euler_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, vc, vu, n, cfg, dt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cfg_slg_euler(float* x, const float* vc, const float* vcs, const float* vu, int64_t n, float cfg,
+                                 float slg, float sigma, float sigma_next, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const float dt = sigma_next - sigma;
+  int64_t blocks = ((n >> 2) + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  cfg_slg_euler_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, vc, vcs, vu, n, cfg, slg, dt);
   return cudaGetLastError();
 }
 

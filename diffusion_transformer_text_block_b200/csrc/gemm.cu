@@ -157,7 +157,7 @@ __device__ __forceinline__ void epi_resid_tma(const EpiParams& ep, const CUtenso
 
 // Token index (within its branch) of a row of the packed [branch; tokens] activations.
 __device__ __forceinline__ int token_of_row(const EpiParams& ep, int row) {
-  if (ep.split_rows > 0) return row >= ep.split_rows ? row - ep.split_rows : row;
+  if (ep.split_rows > 0 && row >= ep.split_rows) return row - ep.split_rows;
   return row % ep.n_tok;
 }
 

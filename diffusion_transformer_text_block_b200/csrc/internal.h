@@ -37,8 +37,9 @@ struct EpiParams {
   const float2* rope = nullptr;      // kEpiQkv: [64, rope_stride] (cos, sin), pair-major
   int rope_stride = 0;               // kEpiQkv: tokens per pair row of the RoPE table
   int n_tok = 0;                     // tokens per branch (of the first branch when split_rows > 0)
-  int split_rows = 0;                // kEpiQkv, two branches of different lengths: rows >= split_rows
-                                     // belong to the second branch (token = row - split_rows)
+  int split_rows = 0;                // kEpiQkv, a last branch of another length: rows >= split_rows
+                                     // belong to it (token = row - split_rows); rows below are
+                                     // branches of n_tok tokens (token = row % n_tok)
   int hidden = 0;                    // D
   int n_branch = 0;                  // kEpiEmbed: branches written
   int n_img = 0, grid_w = 0, lat_h8 = 0, lat_w8 = 0;  // kEpiOut
@@ -88,6 +89,10 @@ cudaError_t launch_cfg_euler(float* x, const float* vc, const float* vu, int64_t
                              float sigma_next, cudaStream_t s);
 
 cudaError_t launch_noise(float* x, int64_t n, uint64_t seed, cudaStream_t s);
+
+// Three-pass SLG step: x += (sigma_next - sigma) * (vu + cfg (vc - vu) + slg (vc - vcs)), FP32.
+cudaError_t launch_cfg_slg_euler(float* x, const float* vc, const float* vcs, const float* vu, int64_t n, float cfg,
+                                 float slg, float sigma, float sigma_next, cudaStream_t s);
 
 // sc[t, :] = SiLU(W2 SiLU(W1 sinusoid(1000 ts[t]) + b1) + b2), t < T.
 cudaError_t launch_conditioning(const bf16* w1, const bf16* b1, const bf16* w2, const bf16* b2, const float* ts,

@@ -273,12 +273,20 @@ typedef struct moss_sample_options {
    * the last full call.  The first step, and a step whose number of branches differs from the
    * last full call's (CFG truncation), always runs in full. */
   double step_cache_threshold;
+  /* Three-pass skip-layer guidance ([SGL-MOSS] 3: three-pass SLG adds a skipped conditional
+   * prediction; the pages give no formula, so this follows the library's reading): > 0 turns
+   * it on, 0 (the default) keeps the two-pass recipe.  On a CFG step inside the
+   * [slg_start, slg_stop] window a third pass runs the conditional branch with
+   * uncond_skip_layers left out (v_cs), and v = v_u + cfg (v_c - v_u) + slg_scale (v_c - v_cs)
+   * in FP32.  Needs max_batch >= 3.  Outside the window, and on truncated steps, two-pass. */
+  double slg_scale;
   int* cached_out;    /* optional HOST int [steps]: 1 where the step reused the cache, else 0 */
   float* change_out;  /* optional HOST float [steps]: the change measured at the step, NaN where
                          there was no full call to compare with (or the cache is off) */
 } moss_sample_options;
 
-/* Defaults: cfg_truncation = 1, step_cache_threshold = 0, no outputs; struct_size as given. */
+/* Defaults: cfg_truncation = 1, step_cache_threshold = 0, slg_scale = 0, no outputs; struct_size
+ * as given. */
 void moss_sample_options_init(moss_sample_options* opt, uint32_t struct_size);
 
 /* moss_sample with the accelerators of `opt` (NULL = defaults, identical to moss_sample).
@@ -286,7 +294,8 @@ void moss_sample_options_init(moss_sample_options* opt, uint32_t struct_size);
  * to choose the step's path) and, on first use, allocates two FP32 buffers of
  * max_batch x max_tokens x hidden owned by the model (freed by moss_model_free).
  * Errors: as moss_sample; MOSS_ERR_ABI_MISMATCH when struct_size is not this version's;
- * MOSS_ERR_INVALID_ARGUMENT for cfg_truncation outside [0, 1] or a negative or NaN threshold;
+ * MOSS_ERR_INVALID_ARGUMENT for cfg_truncation outside [0, 1], a negative or NaN threshold or
+ * slg_scale, slg_scale > 0 with cfg != 1 on a model with max_batch < 3;
  * MOSS_ERR_OOM when the cache buffers cannot be allocated. */
 int moss_sample_ex(moss_model* m, int steps, float cfg, double shift, uint64_t seed,
                    const int* uncond_skip_layers, int n_skip, double slg_start, double slg_stop,

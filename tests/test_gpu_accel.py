@@ -14,6 +14,8 @@ import numpy as np
 import pytest
 import torch
 
+import diffusion_transformer_text_block_b200 as moss
+
 import oracle.moss_oracle as o
 from tests.gpu_common import assert_no_device_error, make_model, psnr
 from synth import TINY, make_text
@@ -118,5 +120,45 @@ def test_step_cache_threshold_zero_equals_moss_sample_bitwise():
     a, cached, _ = _gpu(model, tc, tu, 4, step_cache_threshold=0.0)
     b = model.sample(tc.cuda(), tu.cuda(), 64, 64, steps=4, cfg=3.0, shift=5.0, seed=0, uncond_skip_layers=[1])
     assert np.array_equal(a, b.cpu().numpy()) and not any(cached)
+    model.close()
+    assert_no_device_error()
+
+
+# Three-pass SLG (reading R24: the pages give no formula, so parity is against the oracle's
+# reading, not the pages).
+@pytest.mark.parametrize("n_u", [16, 0, 5])
+def test_three_pass_slg_matches_oracle(n_u):
+    steps = 4
+    model, wg, wn = make_model(TINY, 101, max_tokens=32, max_batch=3, max_latent_hw=64, max_steps=steps)
+    tc = make_text(1, 16, TINY.hidden, 102)[0]
+    tu = make_text(1, max(n_u, 1), TINY.hidden, 103)[0][:n_u].contiguous()
+    out, _, _ = _gpu(model, tc, tu, steps, slg_scale=2.0)
+    ref, _, _ = _oracle(wn, tc, tu, steps, slg_scale=2.0)
+    two, _, _ = _oracle(wn, tc, tu, steps)
+    assert psnr(ref, out) >= 40.0
+    assert psnr(ref, two) < psnr(ref, out)          # the third pass does change the result
+    model.close()
+    assert_no_device_error()
+
+
+def test_three_pass_slg_with_cache_and_truncation():
+    steps = 8
+    model, wg, wn = make_model(TINY, 111, max_tokens=32, max_batch=3, max_latent_hw=64, max_steps=steps)
+    tc = make_text(1, 16, TINY.hidden, 112)[0]
+    tu = make_text(1, 5, TINY.hidden, 113)[0]
+    kw = dict(slg_scale=1.5, step_cache_threshold=0.01, cfg_truncation=0.75, slg_start=0.2, slg_stop=0.6)
+    out, cached, change = _gpu(model, tc, tu, steps, **kw)
+    _check_cache_run(wn, tc, tu, steps, 0.01, out, cached, change, **kw)
+    model.close()
+    assert_no_device_error()
+
+
+def test_three_pass_slg_needs_three_branches_of_workspace():
+    model, wn, tc, tu = _setup(steps=4)            # max_batch 2
+    with pytest.raises(moss.MossError) as e:
+        _gpu(model, tc, tu, 4, slg_scale=2.0)
+    assert e.value.code == 1
+    out, _, _ = _gpu(model, tc, tu, 4, slg_scale=2.0, cfg=1.0)   # no CFG: no third pass, allowed
+    assert np.all(np.isfinite(out))
     model.close()
     assert_no_device_error()

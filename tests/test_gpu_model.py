@@ -173,10 +173,10 @@ def test_block_2048_sampled_rows():
 @pytest.fixture(scope="module")
 def full_model():
     """The 42-block, hidden-3072 DiT with ~5B random BF16 weights (drawn on the GPU), sized for
-    the 1024^2 workload: 4096 image + 512 text tokens per branch, batch 2."""
+    the 1024^2 workload: 4096 image + 512 text tokens per branch, up to 3 branches."""
     from synth import FULL, make_weights
     w = make_weights(FULL, 2, device="cuda")
-    model = moss.Model(FULL, w, max_tokens=4096 + 512, max_batch=2, max_latent_hw=128 * 128, max_steps=2)
+    model = moss.Model(FULL, w, max_tokens=4096 + 512, max_batch=3, max_latent_hw=128 * 128, max_steps=2)
     yield model, w
     model.close()
 
@@ -300,4 +300,30 @@ def test_full_accelerators(full_model):
     torch.cuda.synchronize()
     assert cached == [False, True] and 0.0 < change[1] < 1.0
     assert torch.isfinite(cache).all() and not torch.equal(cache, plain)
+    assert_no_device_error()
+
+
+def test_full_three_pass_slg(full_model):
+    """1024^2, one step from the seed's noise, three-pass SLG (reading R24) with a 77-token
+    negative prompt: the packed three-branch call equals three single-branch forwards combined
+    in FP32.  (One step only: a second step would feed the two results' last-ulp differences
+    through the BF16 patch embedding, which magnifies them.)"""
+    from synth import FULL
+    model, w = full_model
+    tc = make_text(1, 512, FULL.hidden, 41, device="cuda")[0].contiguous()
+    tu = make_text(1, 77, FULL.hidden, 42, device="cuda")[0].contiguous()
+    out, _, _ = model.sample_accelerated(tc, tu, 1024, 1024, steps=1, cfg=3.0, shift=5.0, seed=11,
+                                         uncond_skip_layers=[22], slg_start=0.0, slg_stop=1.0, slg_scale=2.0)
+    x = torch.empty(128, 128, 32, device="cuda")
+    moss.init_noise(x, 11)
+    sig = o.sigma_schedule(1, 5.0)
+    t = float(sig[0])
+    vc = model.forward(x, tc[None], 1024, 1024, t, skip_layers=[[]]).clone()[0]
+    vcs = model.forward(x, tc[None], 1024, 1024, t, skip_layers=[[22]]).clone()[0]
+    vu = model.forward(x, tu[None], 1024, 1024, t, skip_layers=[[22]]).clone()[0]
+    v = vu + 3.0 * (vc - vu) + 2.0 * (vc - vcs)
+    ref = x + (float(np.float32(sig[1])) - float(np.float32(sig[0]))) * v
+    torch.cuda.synchronize()
+    assert rel_l2(out.cpu().numpy(), ref.cpu().numpy()) <= 1e-6
+    assert rel_l2(out.cpu().numpy(), x.cpu().numpy()) > 1e-2      # the step moved the latent
     assert_no_device_error()
