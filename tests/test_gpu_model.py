@@ -327,3 +327,33 @@ def test_full_three_pass_slg(full_model):
     assert rel_l2(out.cpu().numpy(), ref.cpu().numpy()) <= 1e-6
     assert rel_l2(out.cpu().numpy(), x.cpu().numpy()) > 1e-2      # the step moved the latent
     assert_no_device_error()
+
+
+@pytest.mark.parametrize("h,w", [(64, 128), (128, 48), (48, 80)])
+def test_forward_tiny_non_square_matches_oracle(h, w):
+    """Non-square images: the patch grid's rows and columns enter the RoPE positions, the patch
+    order and the unpatchify differently, so a transposed index shows up here."""
+    gh, gw = h // 16, w // 16
+    model, wg, wn = make_model(TINY, 131, max_tokens=gh * gw + 16, max_latent_hw=(h // 8) * (w // 8))
+    lat = make_latent(h // 8, w // 8, 132)
+    txt = make_text(2, 16, TINY.hidden, 133)
+    v = model.forward(lat.cuda(), txt.cuda(), h, w, 0.6, skip_layers=[[], [1]])
+    torch.cuda.synchronize()
+    ref = o.dit_forward(lat.numpy(), txt.double().numpy(), 0.6, [(), (1,)], wn, TINY.heads)
+    for b in range(2):
+        assert rel_l2(v.cpu().numpy()[b], ref[b]) <= 1e-2
+    model.close()
+    assert_no_device_error()
+
+
+def test_sample_tiny_non_square_psnr():
+    model, wg, wn = make_model(TINY, 141, max_tokens=4 * 8 + 16, max_latent_hw=8 * 16, max_steps=4)
+    tc = make_text(1, 16, TINY.hidden, 142)[0]
+    tu = make_text(1, 16, TINY.hidden, 143)[0]
+    out = model.sample(tc.cuda(), tu.cuda(), 64, 128, steps=4, cfg=3.0, shift=5.0, seed=2, uncond_skip_layers=[1])
+    torch.cuda.synchronize()
+    ref = o.sample(wn, TINY.heads, 64, 128, tc.double().numpy(), tu.double().numpy(), steps=4, cfg=3.0, shift=5.0,
+                   seed=2, uncond_skip_layers=(1,))
+    assert psnr(ref, out.cpu().numpy()) >= 40.0
+    model.close()
+    assert_no_device_error()
