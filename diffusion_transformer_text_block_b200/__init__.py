@@ -89,6 +89,7 @@ _SIGS = {
                             ctypes.POINTER(SampleOptions), _P, _P]),
     "moss_device_status": (_I, [_I]),
     "moss_profile_enable": (_I, [_P, _I]),
+    "moss_profile_enable_classes": (_I, [_P, ctypes.c_uint]),
     "moss_profile_read": (_I, [_P, _I, ctypes.POINTER(_I64), ctypes.POINTER(_D)]),
     "moss_launch_count": (_I64, [_I]),
     "moss_op_gemm_bf16": (_I, [_P, _P, _P, _I, _I, _I, _P]),
@@ -401,6 +402,13 @@ class Model:
 
     def profile_enable(self, enable: bool = True):
         _check(lib().moss_profile_enable(self._h, 1 if enable else 0))
+
+    def profile_enable_classes(self, classes):
+        """Time only the launches of the named kernel classes (KERNEL_CLASSES names)."""
+        mask = 0
+        for c in classes:
+            mask |= 1 << KERNEL_CLASSES.index(c)
+        _check(lib().moss_profile_enable_classes(self._h, mask))
 
     def profile_read(self) -> dict:
         out = {}

@@ -223,6 +223,7 @@ struct moss_model {
   CUtensorMap tm_img, tm_out;
   // profiling
   bool prof = false;
+  unsigned prof_mask = 0xFFFFFFFFu;  // classes timed while prof is on
   std::vector<cudaEvent_t> events;
   size_t next_event = 0;
   std::vector<ProfRec> recs;
@@ -258,9 +259,9 @@ bool build_block_maps(int D, int F, int count, const void* wqkv_v, const void* w
   return true;
 }
 
-int prof_begin(moss_model* m, cudaStream_t s) {
+int prof_begin(moss_model* m, int cls, cudaStream_t s) {
   ++g_launches;
-  if (!m || !m->prof) return -1;
+  if (!m || !m->prof || !((m->prof_mask >> cls) & 1u)) return -1;
   if (m->next_event >= m->events.size()) {
     cudaEvent_t e;
     if (cudaEventCreate(&e) != cudaSuccess) return -1;
@@ -285,7 +286,7 @@ void prof_end(moss_model* m, int cls, int i0, cudaStream_t s) {
 
 #define LAUNCH(m, cls, s, call, what)            \
   do {                                           \
-    const int ev_ = prof_begin((m), (s));        \
+    const int ev_ = prof_begin((m), (cls), (s)); \
     cudaError_t e_ = (call);                     \
     prof_end((m), (cls), ev_, (s));              \
     if (e_ != cudaSuccess) return cuda_fail(e_, what); \
@@ -1130,6 +1131,17 @@ int moss_profile_enable(moss_model* m, int enable) {
   g_last_error.clear();
   if (!m) return fail(MOSS_ERR_INVALID_ARGUMENT, "model is NULL");
   m->prof = enable != 0;
+  m->prof_mask = 0xFFFFFFFFu;
+  m->next_event = 0;
+  m->recs.clear();
+  return MOSS_OK;
+}
+
+int moss_profile_enable_classes(moss_model* m, unsigned class_mask) {
+  g_last_error.clear();
+  if (!m) return fail(MOSS_ERR_INVALID_ARGUMENT, "model is NULL");
+  m->prof = class_mask != 0;
+  m->prof_mask = class_mask;
   m->next_event = 0;
   m->recs.clear();
   return MOSS_OK;

@@ -320,6 +320,11 @@ enum {
  * class.  Resets the accumulators. */
 int moss_profile_enable(moss_model* m, int enable);
 
+/* As moss_profile_enable, timing only the launches of the classes whose bit (1 << class) is set
+ * in class_mask (0 disables).  Each timed launch adds two event records to the stream, so a
+ * caller that times the whole step can restrict the timing to the classes it reports. */
+int moss_profile_enable_classes(moss_model* m, unsigned class_mask);
+
 /* Launch count and summed device time (ms) of class `kclass` since the last enable.
  * Synchronises the device. */
 int moss_profile_read(moss_model* m, int kclass, int64_t* launches, double* total_ms);
