@@ -204,24 +204,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdescS = idesc_bf16(128, kKTile, false);
       constexpr uint32_t kIdescO = idesc_bf16(128, 128, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      // Descriptor low words of the operand bases; an offset inside a tile adds (offset >> 4).
+      const uint32_t dq0 = desc_lo(q_addr, 16), dk0 = desc_lo(k_addr, 16), dv0 = desc_lo(v_addr, 2 * kBox);
+      constexpr uint32_t kTileLo = kTileBytes >> 4;
       // S_t(j) = Q_t K_j^T into S_t.
       auto issue_s = [&](int t, int j) {
-        const uint32_t qs = q_addr + t * kTileBytes;
-        const uint32_t ks = k_addr + (j & 1) * kTileBytes;
+        const uint32_t dq = dq0 + t * kTileLo;
+        const uint32_t dk = dk0 + (j & 1) * kTileLo;
+        const uint32_t d = tmem + 128 * t;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // head dim in steps of 16
-          const uint32_t off = (k >> 2) * 2 * kBox + (k & 3) * 32;
-          mma_ss_lo(tmem + 128 * t, desc_lo(qs + off, 16), desc_lo(ks + off, 16), kIdescS, k > 0 ? 1u : 0u);
+          const uint32_t off = ((k >> 2) * 2 * kBox + (k & 3) * 32) >> 4;
+          mma_ss_lo(d, dq + off, dk + off, kIdescS, k > 0 ? 1u : 0u);
         }
         tc_commit(&b_s[t]);
       };
       // O_t += P_t(j) V_j over keys 64 h .. 64 h + 63, P from columns 32 h .. 32 h + 31 of S_t.
       auto issue_pv = [&](int t, int j, int h) {
-        const uint32_t vs = v_addr + (j & 1) * kTileBytes;
+        const uint32_t dv = dv0 + (j & 1) * kTileLo;
+        const uint32_t d = tmem + 256 + 128 * t, p = tmem + 128 * t;
 #pragma unroll
         for (int k = 4 * h; k < 4 * h + 4; ++k)  // keys in steps of 16: P columns advance by 8 words
-          mma_ts_lo(tmem + 256 + 128 * t, tmem + 128 * t + k * 8, desc_lo(vs + k * 16 * 128, 2 * kBox), kIdescO,
-                    (j > 0 || k > 0) ? 1u : 0u);
+          mma_ts_lo(d, p + k * 8, dv + ((k * 16 * 128) >> 4), kIdescO, (j > 0 || k > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(b_q, 0, err, kErrAttnMma, abort_flag) &&
                 mbar_wait(&b_kfull[0], 0, err, kErrAttnMma, abort_flag);
