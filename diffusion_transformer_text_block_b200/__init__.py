@@ -88,6 +88,7 @@ _SIGS = {
     "moss_sample_ex": (_I, [_P, _I, _F, _D, ctypes.c_uint64, _P, _I, _D, _D, _P, _I, _P, _I, _I, _I,
                             ctypes.POINTER(SampleOptions), _P, _P]),
     "moss_device_status": (_I, [_I]),
+    "moss_selftest_wait_timeout": (_I, [_P]),
     "moss_profile_enable": (_I, [_P, _I]),
     "moss_profile_enable_classes": (_I, [_P, ctypes.c_uint]),
     "moss_profile_read": (_I, [_P, _I, ctypes.POINTER(_I64), ctypes.POINTER(_D)]),
@@ -176,6 +177,10 @@ def cfg_euler_step(x, v_c, v_u, cfg: float, sigma: float, sigma_next: float, str
 def init_noise(x, seed: int, stream=None) -> None:
     import torch
     _check(lib().moss_init_noise(_ptr(x, torch.float32, "x"), x.numel(), seed, _stream(stream)))
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    _check(lib().moss_selftest_wait_timeout(_stream(stream)))
 
 
 def device_status(clear: bool = False) -> int:

@@ -1117,6 +1117,15 @@ int moss_sample_ex(moss_model* m, int steps, float cfg, double shift, uint64_t s
   return MOSS_OK;
 }
 
+int moss_selftest_wait_timeout(void* stream) {
+  g_last_error.clear();
+  unsigned* p = device_error_word();
+  if (!p) return fail(MOSS_ERR_CUDA, "could not allocate the device error word");
+  LAUNCH(static_cast<moss_model*>(nullptr), MOSS_K_OTHER, static_cast<cudaStream_t>(stream),
+         launch_wait_probe(p, static_cast<cudaStream_t>(stream)), "wait probe");
+  return MOSS_OK;
+}
+
 int moss_device_status(int clear) {
   unsigned* p = device_error_word();
   if (!p) return -MOSS_ERR_CUDA;

@@ -20,6 +20,7 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
 enum : unsigned {
   kErrGemmProducer = 0x101, kErrGemmMma = 0x102, kErrGemmEpilogue = 0x103,
   kErrAttnProducer = 0x201, kErrAttnMma = 0x202, kErrAttnSoftmax = 0x203,
+  kErrSelfTest = 0x301,  // the bounded-wait self-test's wait, which nothing completes
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

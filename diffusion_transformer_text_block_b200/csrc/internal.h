@@ -113,4 +113,7 @@ cudaError_t launch_change_partials(const float* a, const float* ref, int64_t n, 
 cudaError_t launch_add_inplace(float* x, const float* r, int64_t n, cudaStream_t s);
 cudaError_t launch_sub(float* d, const float* a, const float* b, int64_t n, cudaStream_t s);
 
+// Self-test of the device-side wait limit (records kErrSelfTest after about 2 s).
+cudaError_t launch_wait_probe(unsigned* err, cudaStream_t s);
+
 }  // namespace moss

@@ -310,6 +310,12 @@ int moss_sample_ex(moss_model* m, int steps, float cfg, double shift, uint64_t s
  * the device.  clear != 0 resets it.  Returns the word (>= 0) or -MOSS_ERR_CUDA. */
 int moss_device_status(int clear);
 
+/* Self-test of the device-side wait limit: launches one kernel whose single thread waits on a
+ * barrier phase that nothing completes.  After about 2 s the wait gives up, the kernel records
+ * 0x301 in the device error word (moss_device_status reads it) and returns; the context stays
+ * usable.  Has no counterpart in the pages: it checks the library's own failure path. */
+int moss_selftest_wait_timeout(void* stream);
+
 /* Kernel classes for profiling. */
 enum {
   MOSS_K_GEMM_QKV = 0, MOSS_K_GEMM_OPROJ = 1, MOSS_K_GEMM_GATEUP = 2, MOSS_K_GEMM_DOWN = 3,
