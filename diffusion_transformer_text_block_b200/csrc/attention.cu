@@ -11,19 +11,26 @@
 // Per CTA (384 threads, three warpgroups):
 //   warp 0      TMA: Q_A and Q_B once, then K_j and V_j (128 keys x 128 dims, four 64x64 boxes
 //               with 128-byte swizzle) into two-slot rings.
-//   warp 1      one thread issues S_A(0), S_B(0), then per key tile j:
+//   warp 1      the MMA warp (one elected lane issues): S_A(0), S_B(0), then per key tile j:
 //               PV_A(j) in two halves of 64 keys, S_A(j+1), PV_B(j) likewise, S_B(j+1), so
 //               the tensor pipe works for one tile while the other tile's softmax runs.  The
 //               first half of PV_t(j) starts as soon as the softmax has written the first
 //               half of P_t(j).  S_t(j+1) overwrites the columns PV_t(j) reads P_t(j) from;
 //               tcgen05.mma operations issued by one thread execute in issue order, so no
-//               wait is needed between them.
-//   warps 2, 3  idle (they only lend their registers, below).
+//               wait is needed between them.  This warp waits only on named barriers: an
+//               mbarrier poll (or any shared- or global-memory load) issued behind queued
+//               MMAs stalls until they have been handed to the tensor pipe and leaves it idle
+//               for the poll's latency, about 75 cycles per wait measured.
+//   warp 2      waits (bounded) until V_j and K_{j+1} have landed and passes that on to the
+//               MMA warp through a named barrier, once per step.
+//   warp 3      idle (it only lends its registers, below).
 //   warps 4..7  softmax of tile A, warps 8..11 of tile B; one query row per thread: the row
 //               of 128 scores in one TMEM load, online softmax in the log2 domain with a lazy
-//               rescale of O (only when the running maximum grows by more than 2^8).  When
-//               S_t(j) is complete, the commit that signalled it also covers PV_t(j-1), so
-//               O_t is stable for the rescale.  At the end O / l is stored as BF16.
+//               rescale of O (only when the running maximum grows by more than 2^8).  Three in
+//               eight of the exponentials run on the FMA pipe (a cubic), the rest on MUFU: the
+//               MUFU unit alone (16 per clock per SM) needs as many cycles as the tensor pipe.
+//               When S_t(j) is complete, the commit that signalled it also covers PV_t(j-1),
+//               so O_t is stable for the rescale.  At the end O / l is stored as BF16.
 // Registers: the kernel is launched at 168 per thread (384 x 168 = 64512); warps 0..3 give
 // theirs down to 80 and the softmax warpgroups take 208 (128 x 80 + 256 x 208 = 63488), enough
 // for a row of 128 scores plus the packed P without spilling.  The launcher checks the compiled
@@ -82,34 +89,95 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
+// 2^x for a pair of arguments on the FMA pipe (Cody-Waite split x = n + f, n = round(x),
+// f in [-0.5, 0.5]; 2^f by a cubic fitted for minimum relative error, 1.0e-4; 2^n added to the
+// exponent field).  Arguments below -126 are clamped there (the result is then < 2^-126).
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t xr = f2_add(x, f2_pack(12582912.0f, 12582912.0f));  // 1.5 * 2^23: rounds to an integer
+  const uint64_t n = f2_add(xr, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);
+  uint64_t p = f2_fma(f2_pack(0.05500893f, 0.05500893f), f, f2_pack(0.24221098f, 0.24221098f));
+  p = f2_fma(p, f, f2_pack(0.69328293f, 0.69328293f));
+  p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
+  float q0, q1, r0, r1;
+  f2_unpack(p, q0, q1);
+  f2_unpack(xr, r0, r1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(r0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(r1) << 23));
+}
+
 // MMA issue with each shared-memory descriptor given as its low word (start address and
 // leading byte offset); the high word (stride 1024 bytes, version 1, 128-byte swizzle) is the
-// same for every operand here and is joined inside the instruction's asm.  Keeping 32-bit
-// values lets the issuing thread run within its small register budget.
+// same for every operand here and is joined inside the instruction's asm.
 constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
 __device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) {
   return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
 }
-__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
-                                          uint32_t accumulate) {
+// Issue forms for a whole warp: one lane, chosen by elect.sync, issues.
+__device__ __forceinline__ void mma_ss_lo_e(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                            uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 ad, bd;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "mov.b64 ad, {%1, %5};\n\t"
       "mov.b64 bd, {%2, %5};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kDescHi)
       : "memory");
 }
-__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
-                                          uint32_t accumulate) {
+__device__ __forceinline__ void mma_ts_lo_e(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
+                                            uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 bd;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "mov.b64 bd, {%2, %5};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kDescHi)
       : "memory");
+}
+__device__ __forceinline__ void tc_commit_e(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
+}
+// Bounded wait taken by a whole warp: every lane polls, the result is warp-uniform.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, unsigned* err, unsigned code,
+                                               volatile int* abort) {
+  const uint32_t a = smem_u32(bar);
+  if (__all_sync(0xffffffffu, mbar_try_wait(a, parity))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(a, parity))) return true;
+    if (__any_sync(0xffffffffu, *abort != 0)) return false;
+    if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitTimeoutNs)) {
+      if ((threadIdx.x & 31) == 0) {
+        atomicCAS(err, 0u, code);
+        *abort = 1;
+      }
+      __syncwarp();
+      return false;
+    }
+  }
+}
+// Named barriers: waiting on one does not stall behind the waiting warp's queued MMAs.  Whole
+// warps only.  Every barrier gets one generation per key step on every path (arrivals are made
+// after an abort too, and the waits before them are bounded), and no side can run a
+// generation ahead of the other: the softmax warps pass kBarS + t before they arrive on
+// kBarP + 2 t + h, and the MMA warp arrives on kBarS + t for step j + 1 only after it has passed
+// both P barriers of step j.  So a named-barrier wait can neither complete without its waiter
+// nor be left short of arrivals.
+constexpr uint32_t kBarKV = 1;   // warp 2 <-> MMA warp rendezvous: V_j and K_{j+1} have landed (64)
+constexpr uint32_t kBarP = 2;    // + 2 t + h: half h of P_t(j) is in TMEM (4 softmax warps arrive, 160)
+constexpr uint32_t kBarS = 6;    // + t: S_t(j) has been issued (the MMA warp arrives, 160)
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_arrive(uint32_t id, uint32_t n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -127,7 +195,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* b_vfull = bars + 5;   // [2]
   uint64_t* b_vempty = bars + 7;  // [2]
   uint64_t* b_s = bars + 9;       // [2] S_t(j) complete (tile t), one phase per j
-  uint64_t* b_p = bars + 11;      // [2][2] half h of P_t(j) written (index 2 t + h), one phase per j
   uint64_t* b_done = bars + 15;   // every MMA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -148,7 +215,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&b_vempty[i], 1);
       mbar_init(&b_s[i], 1);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&b_p[i], 4);
     mbar_init(b_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -200,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       constexpr uint32_t kIdescS = idesc_bf16(128, kKTile, false);
       constexpr uint32_t kIdescO = idesc_bf16(128, 128, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
@@ -215,9 +281,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // head dim in steps of 16
           const uint32_t off = ((k >> 2) * 2 * kBox + (k & 3) * 32) >> 4;
-          mma_ss_lo(d, dq + off, dk + off, kIdescS, k > 0 ? 1u : 0u);
+          mma_ss_lo_e(d, dq + off, dk + off, kIdescS, k > 0 ? 1u : 0u);
         }
-        tc_commit(&b_s[t]);
+        tc_commit_e(&b_s[t]);
       };
       // O_t += P_t(j) V_j over keys 64 h .. 64 h + 63, P from columns 32 h .. 32 h + 31 of S_t.
       auto issue_pv = [&](int t, int j, int h) {
@@ -225,60 +291,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d = tmem + 256 + 128 * t, p = tmem + 128 * t;
 #pragma unroll
         for (int k = 4 * h; k < 4 * h + 4; ++k)  // keys in steps of 16: P columns advance by 8 words
-          mma_ts_lo(d, p + k * 8, dv + ((k * 16 * 128) >> 4), kIdescO, (j > 0 || k > 0) ? 1u : 0u);
+          mma_ts_lo_e(d, p + k * 8, dv + ((k * 16 * 128) >> 4), kIdescO, (j > 0 || k > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(b_q, 0, err, kErrAttnMma, abort_flag) &&
-                mbar_wait(&b_kfull[0], 0, err, kErrAttnMma, abort_flag);
+      const bool ok = mbar_wait_warp(b_q, 0, err, kErrAttnMma, abort_flag) &&
+                      mbar_wait_warp(&b_kfull[0], 0, err, kErrAttnMma, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
-        tc_commit(&b_kempty[0]);
+        tc_commit_e(&b_kempty[0]);
       }
-      for (int j = 0; j < nkv && ok; ++j) {
-        const uint32_t use = (j >> 1) & 1;
+      named_arrive(kBarS + 0, 160);
+      named_arrive(kBarS + 1, 160);
+      // Every named-barrier wait below is matched by arrivals the other warps make on every
+      // step, also after an abort (their own waits are bounded), so none of them can hang.
+      for (int j = 0; j < nkv; ++j) {
         const bool more = j + 1 < nkv;
         const int nslot = (j + 1) & 1;
-        const uint32_t nuse = ((j + 1) >> 1) & 1;
-        // tile A: the operands that are ready first, then the two halves of P_A(j)
-        if (!mbar_wait(&b_vfull[j & 1], use, err, kErrAttnMma, abort_flag) ||
-            (more && !mbar_wait(&b_kfull[nslot], nuse, err, kErrAttnMma, abort_flag)) ||
-            !mbar_wait(&b_p[0], j & 1, err, kErrAttnMma, abort_flag)) {
-          ok = false;
-          break;
+        named_sync(kBarKV, 64);
+        // tile A: the two halves of P_A(j)
+        named_sync(kBarP + 0, 160);
+        if (ok) {
+          tc_fence_after();
+          issue_pv(0, j, 0);
         }
-        tc_fence_after();
-        issue_pv(0, j, 0);
-        if (!mbar_wait(&b_p[1], j & 1, err, kErrAttnMma, abort_flag)) {
-          ok = false;
-          break;
+        named_sync(kBarP + 1, 160);
+        if (ok) {
+          tc_fence_after();
+          issue_pv(0, j, 1);
+          if (more) issue_s(0, j + 1);
         }
-        tc_fence_after();
-        issue_pv(0, j, 1);
-        if (more) issue_s(0, j + 1);
+        if (more) named_arrive(kBarS + 0, 160);
         // tile B
-        if (!mbar_wait(&b_p[2], j & 1, err, kErrAttnMma, abort_flag)) {
-          ok = false;
-          break;
+        named_sync(kBarP + 2, 160);
+        if (ok) {
+          tc_fence_after();
+          issue_pv(1, j, 0);
         }
-        tc_fence_after();
-        issue_pv(1, j, 0);
-        if (!mbar_wait(&b_p[3], j & 1, err, kErrAttnMma, abort_flag)) {
-          ok = false;
-          break;
+        named_sync(kBarP + 3, 160);
+        if (ok) {
+          tc_fence_after();
+          issue_pv(1, j, 1);
+          tc_commit_e(&b_vempty[j & 1]);
+          if (more) {
+            issue_s(1, j + 1);
+            tc_commit_e(&b_kempty[nslot]);
+          }
         }
-        tc_fence_after();
-        issue_pv(1, j, 1);
-        tc_commit(&b_vempty[j & 1]);
-        if (more) {
-          issue_s(1, j + 1);
-          tc_commit(&b_kempty[nslot]);
-        }
+        if (more) named_arrive(kBarS + 1, 160);
       }
-      tc_commit(b_done);
+      tc_commit_e(b_done);
+      const uint32_t a = smem_u32(b_done);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(smem_u32(b_done), 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      while (!__all_sync(0xffffffffu, mbar_try_wait(a, 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
+    }
+  } else if (warp == 2) {
+    // Forwards the landing of V_j and K_{j+1} to the MMA warp, once per step, unconditionally
+    // (a rendezvous: neither side can run a step ahead).
+    for (int j = 0; j < nkv; ++j) {
+      mbar_wait_warp(&b_vfull[j & 1], (j >> 1) & 1, err, kErrAttnMma, abort_flag);
+      if (j + 1 < nkv) mbar_wait_warp(&b_kfull[(j + 1) & 1], ((j + 1) >> 1) & 1, err, kErrAttnMma, abort_flag);
+      named_sync(kBarKV, 64);
     }
   }
   } else {
@@ -294,10 +368,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      ok = mbar_wait(&b_s[t], j & 1, err, kErrAttnSoftmax, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {  // warp-uniform: TMEM accesses are .sync.aligned
-        ok = false;
-        break;
+      // The MMA warp has issued S_t(j) (and passed both P_t(j-1) barriers): this warp cannot
+      // arrive on a P barrier a generation ahead of the MMA warp.
+      named_sync(kBarS + t, 160);
+      if (ok) ok = mbar_wait(&b_s[t], j & 1, err, kErrAttnSoftmax, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);  // warp-uniform: TMEM accesses are .sync.aligned
+      if (!ok) {  // after an abort: only the arrivals the MMA warp waits for
+        named_arrive(kBarP + 2 * t, 160);
+        named_arrive(kBarP + 2 * t + 1, 160);
+        continue;
       }
       tc_fence_after();
       const int kvalid = n_tok - j * kKTile;  // keys of this step inside the sequence
@@ -350,8 +429,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[64 * c + 2 * i]), __uint_as_float(sr[64 * c + 2 * i + 1])),
                              scale2, negm2),
                       x0, x1);
-            p0 = exp2_approx(x0);
-            p1 = exp2_approx(x1);
+            if ((i & 7) == 1 || (i & 7) == 4 || (i & 7) == 6) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = exp2_approx(x0);
+              p1 = exp2_approx(x1);
+            }
             acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(p0, p1));
             pk[i] = pack_bf16x2(p0, p1);
           }
@@ -369,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st32(tS + 32 * c, pk);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&b_p[2 * t + c]);
+        named_arrive(kBarP + 2 * t + c, 160);
       }
       float a0, a1, b0, b1;
       f2_unpack(acc2[0], a0, a1);
