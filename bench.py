@@ -139,7 +139,7 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], 0.0, set()
+        sm, mx, reasons, watts = [], 0.0, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -150,12 +150,19 @@ class ClockSampler:
                 mx = max(mx, float(parts[1]))
             except ValueError:
                 continue
+            try:
+                watts.append(float(parts[2]))
+            except ValueError:
+                pass
             for name, val in zip(names, parts[3:7]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
         if not sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        if watts:
+            out["power_w"] = statistics.median(watts)  # median board power while timing
+        return out
 
 
 def cpu_baseline(seconds_hint=True):
