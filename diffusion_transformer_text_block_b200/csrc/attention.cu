@@ -44,7 +44,7 @@ namespace moss {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kRegsLow = 80;    // warps 0..3 after setmaxnreg.dec
+constexpr int kRegsLow = 80;    // warps 0..3 after setmaxnreg.dec (TMA, MMA, K/V forwarding, idle)
 constexpr int kRegsHigh = 208;  // warps 4..11 after setmaxnreg.inc
 constexpr int kQTile = 128;                     // queries per tile (two tiles per CTA)
 constexpr int kKTile = 128;                     // keys per step
@@ -195,8 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* b_vfull = bars + 5;   // [2]
   uint64_t* b_vempty = bars + 7;  // [2]
   uint64_t* b_s = bars + 9;       // [2] S_t(j) complete (tile t), one phase per j
-  uint64_t* b_done = bars + 15;   // every MMA complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* b_done = bars + 11;   // every MMA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
