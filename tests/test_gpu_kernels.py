@@ -38,7 +38,8 @@ def test_gemm_bf16(M, N, K):
 
 
 @pytest.mark.parametrize("B,N,H,qscale", [(1, 32, 2, 1.0), (2, 200, 2, 1.0), (2, 384, 3, 1.0), (1, 520, 2, 4.0),
-                                          (2, 1, 1, 1.0), (1, 300, 1, 32.0)])
+                                          (2, 1, 1, 1.0), (1, 300, 1, 32.0), (1, 129, 1, 1.0), (1, 255, 1, 1.0),
+                                          (2, 257, 1, 1.0), (1, 511, 2, 1.0)])
 def test_attention(B, N, H, qscale):
     """Against the oracle; qscale 32 spreads a row's scores over several hundred (log2 units), so
     exponent arguments fall below -126, where the kernel's polynomial exponentials clamp."""
