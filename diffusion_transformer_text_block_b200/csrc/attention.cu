@@ -25,7 +25,9 @@
 //               MMA warp through a named barrier, once per step.
 //   warp 3      idle (it only lends its registers, below).
 //   warps 4..7  softmax of tile A, warps 8..11 of tile B; one query row per thread: the row
-//               of 128 scores in one TMEM load, online softmax in the log2 domain with a lazy
+//               of 128 scores in one TMEM load for the maximum, the second half's 64 scores
+//               loaded again (still in TMEM) once the first P half is handed over, which frees
+//               registers for more exponentials in flight; online softmax in the log2 domain with a lazy
 //               rescale of O (only when the running maximum grows by more than 2^8).  Three in
 //               eight of the exponentials run on the FMA pipe (a cubic), the rest on MUFU: the
 //               MUFU unit alone (16 per clock per SM) needs as many cycles as the tensor pipe.
@@ -61,6 +63,16 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* tm, u
   for (int h = 0; h < 2; ++h)
 #pragma unroll
     for (int r = 0; r < 2; ++r) tma_load_3d(dst + h * 2 * kBox + r * kBox, tm, bar, x + 64 * h, y + 64 * r, b);
+}
+
+// 32 lanes x 64 columns of 32-bit TMEM words, waiting for completion in the same statement.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
 }
 
 // Packed FP32 pairs: one instruction performs the operation on both halves.
@@ -178,6 +190,43 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t n) {
 }
 __device__ __forceinline__ void named_arrive(uint32_t id, uint32_t n) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// P half c of a key step: exponentials of its 64 scores sv against the maximum m (three in eight
+// of the pairs on the FMA pipe; keys at or past kvalid get P = 0 when the step is not full), BF16
+// pairs into TMEM at tS + 32 c, row sums into acc2; then the MMA warp is told.
+__device__ __forceinline__ void p_half(const uint32_t (&sv)[64], int c, bool full, int kvalid, float m,
+                                       float scale_log2, uint64_t scale2, uint64_t negm2, uint32_t tS, uint32_t bar,
+                                       uint64_t (&acc2)[2]) {
+  uint32_t pk[32];
+  if (full) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float x0, x1, p0, p1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), scale2, negm2), x0, x1);
+      if ((i & 7) == 1 || (i & 7) == 4 || (i & 7) == 6) {
+        exp2_poly2(x0, x1, p0, p1);
+      } else {
+        p0 = exp2_approx(x0);
+        p1 = exp2_approx(x1);
+      }
+      acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(p0, p1));
+      pk[i] = pack_bf16x2(p0, p1);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int k0 = 64 * c + 2 * i;
+      const float p0 = k0 < kvalid ? exp2_approx(fmaf(__uint_as_float(sv[2 * i]), scale_log2, -m)) : 0.f;
+      const float p1 = k0 + 1 < kvalid ? exp2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), scale_log2, -m)) : 0.f;
+      acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(p0, p1));
+      pk[i] = pack_bf16x2(p0, p1);
+    }
+  }
+  tmem_st32(tS + 32 * c, pk);
+  tc_fence_before();
+  __syncwarp();
+  named_arrive(bar, 160);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -419,41 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
       const uint64_t negm2 = f2_pack(-m_run, -m_run);
       uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[32];
-        if (full) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float x0, x1, p0, p1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[64 * c + 2 * i]), __uint_as_float(sr[64 * c + 2 * i + 1])),
-                             scale2, negm2),
-                      x0, x1);
-            if ((i & 7) == 1 || (i & 7) == 4 || (i & 7) == 6) {
-              exp2_poly2(x0, x1, p0, p1);
-            } else {
-              p0 = exp2_approx(x0);
-              p1 = exp2_approx(x1);
-            }
-            acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(p0, p1));
-            pk[i] = pack_bf16x2(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int k0 = 64 * c + 2 * i;
-            const float p0 = k0 < kvalid ? exp2_approx(fmaf(__uint_as_float(sr[k0]), scale_log2, -m_run)) : 0.f;
-            const float p1 =
-                k0 + 1 < kvalid ? exp2_approx(fmaf(__uint_as_float(sr[k0 + 1]), scale_log2, -m_run)) : 0.f;
-            acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(p0, p1));
-            pk[i] = pack_bf16x2(p0, p1);
-          }
-        }
-        tmem_st32(tS + 32 * c, pk);
-        tc_fence_before();
-        __syncwarp();
-        named_arrive(kBarP + 2 * t + c, 160);
-      }
+      p_half(reinterpret_cast<const uint32_t(&)[64]>(sr[0]), 0, full, kvalid, m_run, scale_log2, scale2, negm2, tS,
+             kBarP + 2 * t, acc2);
+      // Keys 64..127 are still in TMEM (P occupies columns 0..63): reloading them lets their
+      // registers go free during the first half.
+      uint32_t s1[64];
+      tmem_ld64(tS + 64, s1);
+      p_half(s1, 1, full, kvalid, m_run, scale_log2, scale2, negm2, tS, kBarP + 2 * t + 1, acc2);
       float a0, a1, b0, b1;
       f2_unpack(acc2[0], a0, a1);
       f2_unpack(acc2[1], b0, b1);
