@@ -344,8 +344,15 @@ int moss_op_gemm_bf16(const void* a, const void* b, float* c, int M, int N, int 
 
 /* Joint attention of one block ([MI] What works: exact attention), on the fused
  * projection layout: qkv device BF16 [batch, N, 3*heads*128] (q | k | v, head h at
- * columns h*128 of each part, q and k already normalised and rotated); o device BF16
- * [batch, N, heads*128] = softmax(q k^T / sqrt(128)) v per head. */
+ * columns h*128 of each part, q and k already normalised and rotated; 16-byte aligned);
+ * o device BF16 [batch, N, heads*128] = softmax(q k^T / sqrt(128)) v per head, no mask.
+ * Numerics: FP32 scores and softmax statistics, P rounded to BF16 for the P V product,
+ * exponentials base 2 (3/8 of them by a cubic with relative error <= 1.0e-4), O
+ * normalised in FP32 and rounded to BF16.  N >= 1, any length (keys and queries past N are
+ * masked).  Errors: MOSS_ERR_INVALID_ARGUMENT for a null or unaligned pointer or batch,
+ * n_tok or heads below 1,
+ * MOSS_ERR_CUDA if the launch fails; a device-side wait that gives up after 2 s records
+ * MOSS_ERR_TIMEOUT's code in the word moss_device_status reads (the kernel then ends). */
 int moss_op_attention(const void* qkv, void* o, int batch, int n_tok, int heads, void* stream);
 
 /* LN-modulate: h[r,:] = BF16(LN(x[r,:]) * (1 + scale) + shift), eps 1e-6, biased
