@@ -350,9 +350,9 @@ int moss_op_gemm_bf16(const void* a, const void* b, float* c, int M, int N, int 
  * exponentials base 2 (3/8 of them by a cubic with relative error <= 1.0e-4), O
  * normalised in FP32 and rounded to BF16.  N >= 1, any length (keys and queries past N are
  * masked).  Errors: MOSS_ERR_INVALID_ARGUMENT for a null or unaligned pointer or batch,
- * n_tok or heads below 1,
- * MOSS_ERR_CUDA if the launch fails; a device-side wait that gives up after 2 s records
- * MOSS_ERR_TIMEOUT's code in the word moss_device_status reads (the kernel then ends). */
+ * n_tok or heads below 1; MOSS_ERR_CUDA if the launch fails.  A device-side wait that gives
+ * up after 2 s sets the device error word (0x201 producer, 0x202 MMA, 0x203 softmax; read
+ * with moss_device_status) and the kernel still ends. */
 int moss_op_attention(const void* qkv, void* o, int batch, int n_tok, int heads, void* stream);
 
 /* LN-modulate: h[r,:] = BF16(LN(x[r,:]) * (1 + scale) + shift), eps 1e-6, biased
