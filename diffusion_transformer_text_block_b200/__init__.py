@@ -89,6 +89,7 @@ _SIGS = {
                             ctypes.POINTER(SampleOptions), _P, _P]),
     "moss_device_status": (_I, [_I]),
     "moss_selftest_wait_timeout": (_I, [_P]),
+    "moss_selftest_attention_timeout": (_I, [_P, _P, _I, _I, _I, _I, _P]),
     "moss_profile_enable": (_I, [_P, _I]),
     "moss_profile_enable_classes": (_I, [_P, ctypes.c_uint]),
     "moss_profile_read": (_I, [_P, _I, ctypes.POINTER(_I64), ctypes.POINTER(_D)]),
@@ -181,6 +182,17 @@ def init_noise(x, seed: int, stream=None) -> None:
 
 def selftest_wait_timeout(stream=None) -> None:
     _check(lib().moss_selftest_wait_timeout(_stream(stream)))
+
+
+def selftest_attention_timeout(qkv, heads: int, step: int, stream=None):
+    """Attention with one CTA's V tile for key `step` never loaded (the failure-path self-test);
+    returns the (meaningless) output tensor."""
+    import torch
+    B, N, _ = qkv.shape
+    o = torch.empty(B, N, heads * 128, device=qkv.device, dtype=torch.bfloat16)
+    _check(lib().moss_selftest_attention_timeout(_ptr(qkv, torch.bfloat16, "qkv"), o.data_ptr(), B, N, heads, step,
+                                                 _stream(stream)))
+    return o
 
 
 def device_status(clear: bool = False) -> int:

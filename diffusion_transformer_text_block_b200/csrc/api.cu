@@ -1126,6 +1126,22 @@ int moss_selftest_wait_timeout(void* stream) {
   return MOSS_OK;
 }
 
+int moss_selftest_attention_timeout(const void* qkv, void* o, int batch, int n_tok, int heads, int step,
+                                    void* stream) {
+  g_last_error.clear();
+  if (!qkv || !o) return fail(MOSS_ERR_INVALID_ARGUMENT, "qkv and o must not be NULL");
+  if (!aligned16(qkv) || !aligned16(o)) return fail(MOSS_ERR_INVALID_ARGUMENT, "16-byte alignment required");
+  if (batch < 1 || n_tok < 1 || heads < 1) return fail(MOSS_ERR_INVALID_ARGUMENT, "batch, n_tok and heads must be >= 1");
+  if (step < 0 || step >= (n_tok + 127) / 128) return fail(MOSS_ERR_INVALID_ARGUMENT, "step must be a key step of the sequence");
+  unsigned* err = device_error_word();
+  if (!err) return fail(MOSS_ERR_CUDA, "device error word");
+  std::string e;
+  ++g_launches;
+  cudaError_t ce = launch_attention(static_cast<const bf16*>(qkv), static_cast<bf16*>(o), batch, n_tok, heads,
+                                    heads * 128, static_cast<cudaStream_t>(stream), err, &e, step);
+  return ce == cudaSuccess ? MOSS_OK : cuda_fail(ce, e.empty() ? "attention" : e.c_str());
+}
+
 int moss_device_status(int clear) {
   unsigned* p = device_error_word();
   if (!p) return -MOSS_ERR_CUDA;

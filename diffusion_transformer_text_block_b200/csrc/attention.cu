@@ -231,7 +231,7 @@ __device__ __forceinline__ void p_half(const uint32_t (&sv)[64], int c, bool ful
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm, bf16* __restrict__ out, int n_tok, int heads, int hidden,
-                float scale_log2, unsigned* err) {
+                float scale_log2, unsigned* err, int test_skip_v_step) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                        // [2] tiles A, B
@@ -297,6 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&b_kfull[slot], kTileBytes);
         load_tile(sK + slot * kTileBytes, &tm, &b_kfull[slot], xk, j * kKTile, b);
         if (j >= 2 && !mbar_wait(&b_vempty[slot], use ^ 1, err, kErrAttnProducer, abort_flag)) break;
+        // Failure-path self-test only: this V tile never lands, so the waits on it run out.
+        if (j == test_skip_v_step && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) continue;
         v_armed[slot] = static_cast<int>(use);
         mbar_arrive_expect_tx(&b_vfull[slot], kTileBytes);
         load_tile(sV + slot * kTileBytes, &tm, &b_vfull[slot], xv, j * kKTile, b);
@@ -516,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_attention(const bf16* qkv, bf16* o, int batch, int n_tok, int heads, int hidden, cudaStream_t s,
-                             unsigned* err, std::string* emsg) {
+                             unsigned* err, std::string* emsg, int test_skip_v_step) {
   static bool configured = false;
   if (!configured) {
     // setmaxnreg.inc waits until the registers it asks for are free in the CTA's pool (its
@@ -541,7 +543,8 @@ cudaError_t launch_attention(const bf16* qkv, bf16* o, int batch, int n_tok, int
     return cudaErrorInvalidValue;
   const float scale_log2 = 1.4426950408889634f / sqrtf(128.0f);
   dim3 grid((n_tok + 2 * kQTile - 1) / (2 * kQTile), heads, batch);
-  attn_kernel<<<grid, kThreads, kSmemBytes, s>>>(tm, o, n_tok, heads, hidden, scale_log2, err);
+  attn_kernel<<<grid, kThreads, kSmemBytes, s>>>(tm, o, n_tok, heads, hidden, scale_log2, err,
+                                                 test_skip_v_step);
   return cudaGetLastError();
 }
 

@@ -75,8 +75,11 @@ cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& a, const CUtensorMap& b
 // qkv: BF16 [batch, n_tok, 3D] (q | k | v); o: BF16 [batch, n_tok, D].  The launcher builds
 // the kernel's TMA descriptor itself; on a descriptor error it returns cudaErrorInvalidValue
 // with the reason in *emsg.
+// test_skip_v_step >= 0 is the failure-path self-test: the CTA of query block 0, head 0, branch 0
+// does not load V for that key step, so a bounded wait runs out and the kernel ends with the error
+// word set.  -1 in every other call.
 cudaError_t launch_attention(const bf16* qkv, bf16* o, int batch, int n_tok, int heads, int hidden, cudaStream_t s,
-                             unsigned* err, std::string* emsg);
+                             unsigned* err, std::string* emsg, int test_skip_v_step = -1);
 
 // rows of x (FP32, [.., D]) -> h (BF16).  With gather_n_img > 0, output row r reads x row
 // (r / gather_n_img) * gather_n_tok + r % gather_n_img (the image rows of every branch).

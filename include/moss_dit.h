@@ -316,6 +316,15 @@ int moss_device_status(int clear);
  * usable.  Has no counterpart in the pages: it checks the library's own failure path. */
 int moss_selftest_wait_timeout(void* stream);
 
+/* Failure-path self-test of the attention kernel: the same call as moss_op_attention, except that
+ * the CTA of query block 0, head 0, branch 0 never loads V for key step `step` (0 <= step <
+ * ceil(n_tok / 128)).  Its bounded waits run out after 2 s, the device error word reads 0x201 or
+ * 0x202 (whichever wait gave up first), o is not meaningful, and every warp of the kernel still
+ * finishes (the named-barrier arrivals are unconditional); later launches compute normally.
+ * Has no counterpart in the pages. */
+int moss_selftest_attention_timeout(const void* qkv, void* o, int batch, int n_tok, int heads, int step,
+                                    void* stream);
+
 /* Kernel classes for profiling. */
 enum {
   MOSS_K_GEMM_QKV = 0, MOSS_K_GEMM_OPROJ = 1, MOSS_K_GEMM_GATEUP = 2, MOSS_K_GEMM_DOWN = 3,
