@@ -154,14 +154,15 @@ def test_invalid_requests_launch_nothing():
     model.close()
 
 
-def test_block_2048_sampled_rows():
-    """One full-width block at the 2048^2 long-sequence shape (16384 image + 4096 text tokens,
-    batch 2): sampled rows against the oracle's row-restricted block."""
-    gh = gw = 128
+@pytest.mark.parametrize("gh,gw", [(128, 128), (256, 64)])
+def test_block_2048_sampled_rows(gh, gw):
+    """One full-width block at the largest token count the size rule allows (4.2 MP: 16384 image
+    + 4096 text tokens, batch 2), square 2048^2 and the 4096 x 1024 extreme (patch rows up to 255):
+    sampled rows against the oracle's row-restricted block."""
     n_txt = 4096
     model, x, y, lw, mod, ang = _block_case(WIDE1, 45, gh, gw, n_txt, 2, 0.41)
     N = gh * gw + n_txt
-    rows = np.array([0, 127, 128, 16383, 16384, N - 1, 9000])
+    rows = np.array([0, gw - 1, gw, 16383, 16384, N - 1, 9000])
     for b in range(2):
         ref = o.block_forward_rows(x[b], lw, mod, ang, rows, WIDE1.heads)
         assert rel_l2(y[b][rows], ref) <= 1e-2
