@@ -519,8 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_attention(const bf16* qkv, bf16* o, int batch, int n_tok, int heads, int hidden, cudaStream_t s,
                              unsigned* err, std::string* emsg, int test_skip_v_step) {
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};
+  if (!configured_on_device(configured)) {
     // setmaxnreg.inc waits until the registers it asks for are free in the CTA's pool (its
     // threads x the registers per thread at launch), so a split that does not fit would never
     // return: refuse to launch unless the compiled count covers it.
@@ -533,7 +533,7 @@ cudaError_t launch_attention(const bf16* qkv, bf16* o, int batch, int n_tok, int
     }
     e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured = true;
+    mark_configured_on_device(configured);
   }
   if (batch <= 0 || n_tok <= 0) return cudaSuccess;
   // The tensor map is built here, from the same box constants the kernel's shared-memory

@@ -377,10 +377,11 @@ cudaError_t launch_mod_gemv(const bf16* W, const bf16* bias, const float* sc, fl
                             int64_t out_stride, cudaStream_t s) {
   if (R <= 0 || T <= 0) return cudaSuccess;
   const size_t smem = static_cast<size_t>(T) * cdim * sizeof(float);
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(mod_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    configured = true;
+  static std::atomic<uint64_t> configured{0};
+  if (!configured_on_device(configured)) {
+    const cudaError_t e = cudaFuncSetAttribute(mod_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e != cudaSuccess) return e;
+    mark_configured_on_device(configured);
   }
   mod_gemv_kernel<<<(R + 7) / 8, 256, smem, s>>>(W, bias, sc, out, R, cdim, T, out_stride);
   return cudaGetLastError();

@@ -671,12 +671,12 @@ template <int BN, int EPI>
 cudaError_t launch_single(const CUtensorMap& a, const CUtensorMap& b, const EpiParams& ep, cudaStream_t s,
                           unsigned* err) {
   using S = GemmShape<BN>;
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};
+  if (!configured_on_device(configured)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          S::kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured = true;
+    mark_configured_on_device(configured);
   }
   const int tiles = ((ep.M + kBM - 1) / kBM) * ((ep.N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
@@ -689,12 +689,12 @@ template <int EPI>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const EpiParams& ep,
                         cudaStream_t s, unsigned* err) {
   using S = PairShape<EPI>;
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};
+  if (!configured_on_device(configured)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          S::kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured = true;
+    mark_configured_on_device(configured);
   }
   // The residual stream's reduction descriptor is built here from the same box constants the
   // epilogue's staging layout uses.

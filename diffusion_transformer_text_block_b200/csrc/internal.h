@@ -6,9 +6,23 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <string>
 
 namespace moss {
+
+// One-time per-device setup of a kernel (function attributes are set per device): `done` holds
+// one bit per device ordinal.  Two threads may both run the setup the first time; it is
+// idempotent.
+inline bool configured_on_device(const std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  return (done.load(std::memory_order_acquire) >> (dev & 63)) & 1u;
+}
+inline void mark_configured_on_device(std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) done.fetch_or(uint64_t{1} << (dev & 63), std::memory_order_release);
+}
 
 using bf16 = __nv_bfloat16;
 
