@@ -35,9 +35,12 @@
 //               so O_t is stable for the rescale.  At the end O / l is stored as BF16.
 // Registers: the kernel is launched at 168 per thread (384 x 168 = 64512); warps 0..3 give
 // theirs down to 80 and the softmax warpgroups take 208 (128 x 80 + 256 x 208 = 63488), enough
-// for a row of 128 scores plus the packed P without spilling.  The launcher checks the compiled
-// register count against that sum before the first launch.
+// for a row of 128 scores plus the packed P (ptxas reports 8 bytes of spill stores, outside the
+// MMA warp).  The launcher checks the compiled register count against that sum before the first
+// launch.
 // Keys past the sequence end (the TMA fills them with zeros) are masked to -inf.
+// A test-only argument makes one CTA skip a V load so that its bounded waits run out (the
+// library's failure-path self-test); it is -1 in every other launch.
 #include "common.cuh"
 #include "internal.h"
 
