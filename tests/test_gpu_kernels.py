@@ -3,7 +3,8 @@
 Tolerances, from the arithmetic:
   * GEMM: exact BF16 inputs, FP32 accumulation over K -> relative L2 <= 1e-5.
   * attention: P is rounded to BF16 before the PV product and O is stored in BF16
-    (unit roundoff 2^-9 each) -> relative L2 <= 1e-2.
+    (unit roundoff 2^-9 each); 3/8 of the exponentials come from a cubic with relative error
+    <= 1.0e-4, well below that -> relative L2 <= 1e-2.
   * LN-modulate: BF16 output -> relative L2 <= 5e-3.
   * CFG + Euler: FP32, <= 1e-6 relative to the magnitude of the terms (FMA allowed).
   * noise: FP32 Box-Muller on identical integers -> |dz| <= 1e-5 (1 + |z|).
