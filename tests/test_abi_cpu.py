@@ -99,6 +99,14 @@ def test_elementwise_entry_points_check_arguments_without_launching():
     assert lib.moss_op_gemm_bf16(ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), 8, 48, 64, None) == 1
     assert lib.moss_dit_forward(None, 2, None, None, 0, 64, 64, 0.5, None, 0, None, None) == 1
     assert lib.moss_slg_active(50, 50, 0.0, 1.0) == -1
+    a16, b16 = ctypes.c_void_p(4096), ctypes.c_void_p(8192)
+    assert lib.moss_op_attention(None, b16, 1, 128, 1, None) == 1
+    assert lib.moss_op_attention(ctypes.c_void_p(4100), b16, 1, 128, 1, None) == 1          # misaligned
+    assert lib.moss_op_attention(a16, b16, 1, 0, 1, None) == 1
+    # the attention failure-path self-test: the step must be a key step of the sequence
+    assert lib.moss_selftest_attention_timeout(a16, b16, 1, 256, 1, -1, None) == 1
+    assert lib.moss_selftest_attention_timeout(a16, b16, 1, 256, 1, 2, None) == 1          # 2 key steps
+    assert lib.moss_selftest_attention_timeout(None, b16, 1, 256, 1, 0, None) == 1
     assert lib.moss_launch_count(0) == before
 
 
