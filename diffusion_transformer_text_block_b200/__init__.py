@@ -247,9 +247,23 @@ def modulation_noalloc(shape, weights: dict, ts: Sequence[float], out=None, stre
     here (by torch, when not given); the library itself allocates nothing."""
     import torch
     L = weights["mod_w"].shape[0]
-    D = shape.hidden
+    D, C = shape.hidden, shape.c_t
+    stride = L * 6 * D + 2 * D
+    # The library reads these weights and writes len(ts) rows of `stride` floats through raw
+    # pointers; nothing below the C ABI can see a buffer's size, so every shape is checked here.
+    need = {"t_w1": (C, 256), "t_b1": (C,), "t_w2": (C, C), "t_b2": (C,), "mod_w": (L, 6 * D, C),
+            "mod_b": (L, 6 * D), "final_mod_w": (2 * D, C), "final_mod_b": (2 * D,)}
+    for name, want_shape in need.items():
+        if tuple(weights[name].shape) != want_shape:
+            raise MossError(1, f"{name} must have shape {want_shape}, got {tuple(weights[name].shape)}")
+    if out is not None and out.numel() < len(ts) * stride:
+        raise MossError(1, f"out holds {out.numel()} floats; {len(ts)} timesteps need {len(ts) * stride}")
     if out is None:
-        out = torch.empty(len(ts), L * 6 * D + 2 * D, device="cuda", dtype=torch.float32)
+        out = torch.empty(len(ts), stride, device="cuda", dtype=torch.float32)
+    dev = torch.cuda.current_device()
+    for name, t in [("out", out)] + [(k, weights[k]) for k in need]:
+        if t.is_cuda and t.device.index != dev:
+            raise MossError(1, f"{name} is on cuda:{t.device.index}, not on the current device cuda:{dev}")
     cfg = _config_for(shape, L)
     w = Weights()
     lib().moss_weights_init(ctypes.byref(w), ctypes.sizeof(Weights))

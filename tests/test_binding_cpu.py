@@ -74,3 +74,24 @@ def test_every_bound_name_is_declared():
     decls = _declarations()
     for name in moss._SIGS:
         assert name in decls, f"{name} is bound but not declared in the header"
+
+
+def test_modulation_noalloc_checks_buffer_sizes_before_any_call():
+    """The allocation-free entry point writes len(ts) rows of L*6D + 2D floats through a raw
+    pointer: the binding refuses an `out` that is too short, and weights whose shapes do not match
+    the layer count and widths, before it touches the library or a device."""
+    import pytest
+    import torch
+
+    from synth import TINY, make_weights
+
+    w = make_weights(TINY, 1)
+    stride = TINY.layers * 6 * TINY.hidden + 2 * TINY.hidden
+    with pytest.raises(moss.MossError, match="out holds"):
+        moss.modulation_noalloc(TINY, w, [0.5, 0.25], out=torch.empty(2 * stride - 1))
+    bad = dict(w, mod_b=w["mod_b"][:1])
+    with pytest.raises(moss.MossError, match="mod_b must have shape"):
+        moss.modulation_noalloc(TINY, bad, [0.5], out=torch.empty(stride))
+    bad = dict(w, final_mod_w=w["final_mod_w"][:, :128])
+    with pytest.raises(moss.MossError, match="final_mod_w must have shape"):
+        moss.modulation_noalloc(TINY, bad, [0.5], out=torch.empty(stride))

@@ -197,6 +197,154 @@ def test_conditioning_and_modulation_shapes_and_linearity():
                                   w["mod_b"][0])
 
 
+def _T(a):
+    return torch.from_numpy(np.ascontiguousarray(a))
+
+
+def test_conditioning_matches_torch_composition():
+    """The time MLP (InvokeAI MOSS-Image guide, Transformer formats: time-embedding layers; reading
+    R7) as nn.Linear -> SiLU -> nn.Linear on nonzero random weights.  A dropped SiLU, a transposed
+    W1 or W2 (W2 is square, so only the values tell) or a missing bias fails here."""
+    w = numpy_weights(make_weights(TINY, 21))
+    for t in (0.0, 0.37, 0.9):
+        emb = _T(o.timestep_embedding(t))
+        ref = Fnn.linear(Fnn.silu(Fnn.linear(emb, _T(w["t_w1"]), _T(w["t_b1"]))), _T(w["t_w2"]), _T(w["t_b2"]))
+        got = o.conditioning(t, w)
+        np.testing.assert_allclose(got, ref.numpy(), rtol=1e-12, atol=1e-15)
+    # the same MLP with W2 transposed is a different function on these weights
+    wt = dict(w, t_w2=w["t_w2"].T.copy())
+    assert np.abs(o.conditioning(0.37, wt) - o.conditioning(0.37, w)).max() > 1e-3
+
+
+def test_conditioning_closed_form_at_t0():
+    """At t = 0 the sinusoid is [1]*128 + [0]*128, so with W2 = I and b2 = 0 the MLP is
+    SiLU(sum of W1's first 128 columns + b1), written with scipy's logistic function."""
+    from scipy.special import expit
+    w = numpy_weights(make_weights(TINY, 22))
+    C = TINY.c_t
+    w2 = dict(w, t_w2=np.eye(C), t_b2=np.zeros(C))
+    h1 = w["t_w1"][:, :128].sum(axis=1) + w["t_b1"]
+    np.testing.assert_allclose(o.conditioning(0.0, w2), h1 * expit(h1), rtol=1e-12, atol=1e-15)
+
+
+def test_block_modulation_matches_torch_composition():
+    """W_mod SiLU(c) + b_mod (reading R7) against nn.Linear(SiLU(c)); then the SiLU is located by its
+    limits: c -> -inf switches the weights off (only b remains), c -> +inf passes c through."""
+    w = numpy_weights(make_weights(TINY, 23))
+    c = o.conditioning(0.61, w)
+    for l in range(TINY.layers):
+        ref = Fnn.linear(Fnn.silu(_T(c)), _T(w["mod_w"][l]), _T(w["mod_b"][l])).numpy()
+        np.testing.assert_allclose(o.block_modulation(c, w["mod_w"][l], w["mod_b"][l]), ref, rtol=1e-12, atol=1e-15)
+    W, b = w["mod_w"][0], w["mod_b"][0]
+    neg = np.full(TINY.c_t, -60.0)
+    np.testing.assert_allclose(o.block_modulation(neg, W, b), b, rtol=0, atol=1e-20)
+    pos = np.full(TINY.c_t, 60.0)
+    np.testing.assert_allclose(o.block_modulation(pos, W, b), 60.0 * W.sum(axis=1) + b, rtol=1e-12, atol=1e-12)
+
+
+def test_final_layer_matches_torch_composition():
+    """The output layers (InvokeAI guide, Transformer formats; reading R7): [shift_f, scale_f] =
+    Linear(SiLU(c)), then LayerNorm(x) (1 + scale_f) + shift_f, then Linear(out_w, out_b)."""
+    w = numpy_weights(make_weights(TINY, 24))
+    rng = np.random.default_rng(24)
+    D = TINY.hidden
+    x = rng.standard_normal((16, D)) * 2 + 0.5
+    c = o.conditioning(0.44, w)
+    sh, sc = Fnn.linear(Fnn.silu(_T(c)), _T(w["final_mod_w"]), _T(w["final_mod_b"])).chunk(2)
+    y = Fnn.layer_norm(_T(x), (D,), eps=1e-6) * (1 + sc) + sh
+    ref = Fnn.linear(y, _T(w["out_w"]), _T(w["out_b"])).numpy()
+    got = o.final_layer(x, c, w)
+    assert got.shape == (16, 128)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-13)
+    # shift and scale swapped is a different function on these weights
+    y_sw = Fnn.layer_norm(_T(x), (D,), eps=1e-6) * (1 + sh) + sc
+    ref_sw = Fnn.linear(y_sw, _T(w["out_w"]), _T(w["out_b"])).numpy()
+    assert np.abs(got - ref_sw).max() > 1e-3
+
+
+def test_final_layer_scale_minus_one_leaves_the_shift():
+    """With zero modulation weights and bias [shift, -1], the normalised input drops out: every
+    row's output is shift . out_w^T + out_b, whatever x is."""
+    w = numpy_weights(make_weights(TINY, 25))
+    D = TINY.hidden
+    rng = np.random.default_rng(25)
+    shift = rng.standard_normal(D)
+    wz = dict(w, final_mod_w=np.zeros_like(w["final_mod_w"]), final_mod_b=np.concatenate([shift, -np.ones(D)]))
+    x = rng.standard_normal((8, D)) * 3
+    want = shift @ w["out_w"].T + w["out_b"]
+    np.testing.assert_allclose(o.final_layer(x, rng.standard_normal(TINY.c_t), wz), np.broadcast_to(want, (8, 128)),
+                               rtol=1e-12, atol=1e-12)
+
+
+def _torch_forward_skip_all(lat, c, w, gh, gw):
+    """Patch embedding -> final layer -> unpatchify with einops and torch.nn.functional."""
+    D = w["img_w"].shape[0]
+    tok = rearrange(_T(lat), "(h p1) (w p2) c -> (h w) (p1 p2 c)", p1=2, p2=2)
+    img = Fnn.linear(tok, _T(w["img_w"]), _T(w["img_b"]))
+    sh, sc = Fnn.linear(Fnn.silu(_T(c)), _T(w["final_mod_w"]), _T(w["final_mod_b"])).chunk(2)
+    y = Fnn.layer_norm(img, (D,), eps=1e-6) * (1 + sc) + sh
+    v = Fnn.linear(y, _T(w["out_w"]), _T(w["out_b"]))
+    return rearrange(v, "(h w) (p1 p2 c) -> (h p1) (w p2) c", h=gh, w=gw, p1=2, p2=2).numpy()
+
+
+def test_patch_embed_line_matches_torch_composition():
+    """The image embedding of the forward (2x2 patches of the 32-channel latent, windpaint.ai
+    Architecture and specs; reading R10): with every layer skipped, the forward is patch embed ->
+    final layer -> unpatchify, here rebuilt from einops and nn.functional on a non-square latent."""
+    w = numpy_weights(make_weights(TINY, 26))
+    rng = np.random.default_rng(26)
+    lat = rng.standard_normal((8, 12, 32)).astype(np.float32)
+    txt = rng.standard_normal((2, 5, TINY.hidden))
+    v = o.dit_forward(lat, txt, 0.52, [(0, 1), (0, 1)], w, TINY.heads)
+    ref = _torch_forward_skip_all(lat.astype(np.float64), o.conditioning(0.52, w), w, 4, 6)
+    np.testing.assert_allclose(v[0], ref, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(v[1], ref, rtol=1e-11, atol=1e-13)
+
+
+def test_patch_embed_is_local_to_its_patch():
+    """With every layer skipped, tokens do not interact: changing the latent inside the 2x2 patch of
+    token (r, c) changes the velocity in exactly that patch and nowhere else."""
+    w = numpy_weights(make_weights(TINY, 27))
+    rng = np.random.default_rng(27)
+    lat = rng.standard_normal((8, 12, 32)).astype(np.float32)
+    txt = rng.standard_normal((1, 3, TINY.hidden))
+    base = o.dit_forward(lat, txt, 0.3, [(0, 1)], w, TINY.heads)[0]
+    r, c = 2, 5
+    lat2 = lat.copy()
+    lat2[2 * r + 1, 2 * c, 7] += 3.0
+    moved = np.abs(o.dit_forward(lat2, txt, 0.3, [(0, 1)], w, TINY.heads)[0] - base).max(axis=-1) > 0
+    want = np.zeros((8, 12), dtype=bool)
+    want[2 * r:2 * r + 2, 2 * c:2 * c + 2] = True
+    np.testing.assert_array_equal(moved, want)
+
+
+def test_forward_matches_torch_composition():
+    """The whole forward on both branches (one with layer 1 skipped) rebuilt from the torch block
+    composition below, the torch patch embedding and the torch final layer."""
+    w = numpy_weights(make_weights(TINY, 28))
+    rng = np.random.default_rng(28)
+    lat = rng.standard_normal((8, 8, 32)).astype(np.float32)
+    txt = rng.standard_normal((2, 6, TINY.hidden))
+    t = 0.71
+    v = o.dit_forward(lat, txt, t, [(), (1,)], w, TINY.heads)
+    c = _T(o.conditioning(t, w))
+    ang = o.rope_angles(o.token_positions(4, 4, 6))
+    tok = rearrange(_T(lat.astype(np.float64)), "(h p1) (w p2) c -> (h w) (p1 p2 c)", p1=2, p2=2)
+    img = Fnn.linear(tok, _T(w["img_w"]), _T(w["img_b"])).numpy()
+    for b, skip in enumerate([(), (1,)]):
+        x = np.concatenate([img, txt[b]])
+        for l in range(TINY.layers):
+            if l in skip:
+                continue
+            mod = Fnn.linear(Fnn.silu(c), _T(w["mod_w"][l]), _T(w["mod_b"][l])).numpy()
+            x = _torch_block(x, o.layer_weights(w, l), mod, ang, TINY.heads)
+        sh, sc = Fnn.linear(Fnn.silu(c), _T(w["final_mod_w"]), _T(w["final_mod_b"])).chunk(2)
+        y = Fnn.layer_norm(_T(x[:16]), (TINY.hidden,), eps=1e-6) * (1 + sc) + sh
+        vt = Fnn.linear(y, _T(w["out_w"]), _T(w["out_b"]))
+        ref = rearrange(vt, "(h w) (p1 p2 c) -> (h p1) (w p2) c", h=4, w=4, p1=2, p2=2).numpy()
+        np.testing.assert_allclose(v[b], ref, rtol=1e-10, atol=1e-12)
+
+
 # ---------------------------------------------------------------- normalisation
 def test_layer_norm_matches_torch():
     rng = np.random.default_rng(1)
