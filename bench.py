@@ -165,12 +165,9 @@ class ClockSampler:
         return out
 
 
-def cpu_baseline(seconds_hint=True):
-    """The oracle (float64 numpy, as it stands) on one branch-block of the 1024^2 workload:
-    4608 tokens, hidden 3072.  forwards/s = 1 / (42 * block time)."""
-    import numpy as np
-    from threadpoolctl import threadpool_info
-
+def oracle_block_sampler():
+    """One branch-block of the 1024^2 workload (4608 tokens, hidden 3072) in the float64 oracle, as
+    it stands: returns a function that runs it once and returns the seconds it took."""
     from oracle import moss_oracle as o
     from synth import ModelShape, make_residual, make_weights, numpy_weights
 
@@ -181,28 +178,51 @@ def cpu_baseline(seconds_hint=True):
     c = o.conditioning(0.5, wn)
     mod = o.block_modulation(c, wn["mod_w"][0], wn["mod_b"][0])
     lw = o.layer_weights(wn, 0)
-    t0 = time.perf_counter()
-    o.block_forward(x, lw, mod, ang, shape.heads)
-    dt = time.perf_counter() - t0
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    return {"value": 1.0 / (42 * dt), "unit": UNIT, "cores": threads, "kind": "oracle",
+
+    def run_once():
+        t0 = time.perf_counter()
+        o.block_forward(x, lw, mod, ang, shape.heads)
+        return time.perf_counter() - t0
+
+    return run_once
+
+
+def _oracle_threads():
+    from threadpoolctl import threadpool_info
+    return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+
+
+def cpu_baseline(run_once=None):
+    """The oracle on one branch-block of the 1024^2 workload, timed once: forwards/s =
+    1 / (42 * block time)."""
+    run_once = run_once or oracle_block_sampler()
+    dt = run_once()
+    return {"value": 1.0 / (42 * dt), "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
             "sample": f"one branch-block (4608 tokens x 3072, float64) timed once: {dt:.2f} s; "
                       f"forwards/s = 1/(42 x block time)"}
 
 
 def run_reference(args):
+    """The oracle as it stands, on the host cores: each of the --steps timed steps runs one
+    branch-block of the workload (a bounded sample of the step's 83), and the step time is
+    extrapolated from the mean block time.  Rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    steps = max(1, args.steps if args.steps <= 3 else 2)
-    vals = [cpu_baseline()["value"] for _ in range(steps)]
-    cb = cpu_baseline()
-    value = statistics.mean(vals)
+    steps = max(1, args.steps)
+    warm = min(args.warmup, 1)
+    run_once = oracle_block_sampler()
+    for _ in range(warm):
+        run_once()
+    samples = [cpu_baseline(run_once) for _ in range(steps)]
+    value = statistics.mean(s["value"] for s in samples)
+    cb = dict(samples[-1], value=value, sample=REFERENCE_SAMPLE)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": steps, "warmup": 0, "ms_per_step": 2000.0 / value, "higher_is_better": True,
+            "steps": steps, "warmup": warm, "ms_per_step": 2000.0 / value, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": 4096 + N_TXT, "parallelism": "none"},
-            "cpu_baseline": dict(cb, value=value),
+            "extrapolated": True, "timed_per_step": "one branch-block (4608 tokens x 3072)",
+            "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -461,6 +481,9 @@ def main():
     for i in range(args.warmup):
         step(i)
     moss.init_noise(x, 42 + rank)
+    # The warm-up left the schedule's modulation in the model; drop it, so that the first timed
+    # step computes it for the whole schedule as moss_sample does once per image.
+    model.modulation(0.5)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -539,28 +562,28 @@ def main():
     step_flops = sum(fl.values()) * bl / args.steps
     tc_frac = step_flops * args.steps / (ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]
 
-    # end to end through the public API with host buffers
+    # End to end through the C-ABI call with host buffers (moss_denoise_step_host): every step
+    # copies the latent and both prompts from pinned host memory to the device, runs the step and
+    # copies the latent back, all inside the call; the call returns with the result in host memory.
     e2e = None
     if args.e2e_steps > 0:
-        hx = torch.empty_like(x, device="cpu").pin_memory()
+        hx = x.cpu().pin_memory()
         htc = tc.cpu().pin_memory()
         htu = tu.cpu().pin_memory()
-        hx.copy_(x.cpu())
+        model.modulation(0.5)  # as above: the first e2e step computes the schedule's modulation
         torch.cuda.synchronize()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         for i in range(args.e2e_steps):
-            x.copy_(hx, non_blocking=True)
-            tc.copy_(htc, non_blocking=True)
-            tu.copy_(htu, non_blocking=True)
-            step(i)
-            hx.copy_(x, non_blocking=True)
+            model.denoise_step_host(hx, htc, htu, HEIGHT, WIDTH, i % STEPS_PER_IMAGE, STEPS_PER_IMAGE, CFG, SHIFT,
+                                    SKIP, *SLG)
         a1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(a0.elapsed_time(a1), dist if world > 1 else None, "cuda")
         e2e = {"value": job_throughput(args.e2e_steps, world, ems)[0], "unit": UNIT,
-               "h2d_bytes_per_step": x.numel() * 4 + tc.numel() * 4 + tu.numel() * 4,
-               "d2h_bytes_per_step": x.numel() * 4, "steps": args.e2e_steps}
+               "h2d_bytes_per_step": hx.numel() * 4 + htc.numel() * 4 + htu.numel() * 4,
+               "d2h_bytes_per_step": hx.numel() * 4, "steps": args.e2e_steps,
+               "call": "moss_denoise_step_host (pinned host buffers, copies and a stream wait inside the call)"}
 
     model.close()
     if world > 1:

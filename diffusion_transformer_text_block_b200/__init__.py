@@ -80,6 +80,7 @@ _SIGS = {
     "moss_slg_active": (_I, [_I, _I, _D, _D]),
     "moss_init_noise": (_I, [_P, _I64, ctypes.c_uint64, _P]),
     "moss_denoise_step": (_I, [_P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _F, _D, _P, _I, _D, _D, _P]),
+    "moss_denoise_step_host": (_I, [_P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _F, _D, _P, _I, _D, _D, _P]),
     "moss_sample": (_I, [_P, _I, _F, _D, ctypes.c_uint64, _P, _I, _D, _D, _P, _I, _P, _I, _I, _I, _P, _P]),
     "moss_text_weights_init": (None, [ctypes.POINTER(TextWeights), ctypes.c_uint32]),
     "moss_text_refiner_set": (_I, [_P, ctypes.POINTER(TextWeights)]),
@@ -147,6 +148,20 @@ def _ptr(t, dtype=None, name="tensor"):
         raise MossError(1, f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise MossError(1, f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _host_ptr(t, name="tensor"):
+    """Address of a contiguous FP32 CPU tensor (pinned or pageable) for the host-buffer calls."""
+    import torch
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise MossError(1, f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise MossError(1, f"{name} must be contiguous")
+    if t.dtype != torch.float32:
+        raise MossError(1, f"{name} must be torch.float32, got {t.dtype}")
     return t.data_ptr()
 
 
@@ -381,6 +396,25 @@ class Model:
         _check(lib().moss_denoise_step(self._h, _ptr(x, f, "x"), _ptr(text_c, f, "text_c"), text_c.shape[0],
                                        _ptr(text_u, f, "text_u") if text_u is not None else None, n_u, height,
                                        width, step, steps, cfg, shift, arr, n, slg_start, slg_stop, _stream(stream)))
+        return x
+
+    def denoise_step_host(self, x, text_c, text_u, height: int, width: int, step: int, steps: int = 50,
+                          cfg: float = 3.0, shift: float = 5.0, uncond_skip_layers: Sequence[int] = (22,),
+                          slg_start: float = 0.01, slg_stop: float = 1.0, stream=None):
+        """moss_denoise_step_host: x, text_c, text_u are FP32 CPU tensors (pinned for asynchronous
+        copies); x is updated in place and holds the result when the call returns."""
+        nx = (height // 8) * (width // 8) * 32
+        D = self.shape.hidden
+        if x.numel() != nx:
+            raise MossError(1, f"x must hold {nx} floats")
+        n_u = text_u.shape[0] if text_u is not None else 0
+        if text_c.numel() != text_c.shape[0] * D or (text_u is not None and text_u.numel() != n_u * D):
+            raise MossError(1, f"text states must be [n, {D}]")
+        arr, n = _skip_array([list(uncond_skip_layers)])
+        _check(lib().moss_denoise_step_host(self._h, _host_ptr(x, "x"), _host_ptr(text_c, "text_c"), text_c.shape[0],
+                                            _host_ptr(text_u, "text_u") if text_u is not None else None, n_u, height,
+                                            width, step, steps, cfg, shift, arr, n, slg_start, slg_stop,
+                                            _stream(stream)))
         return x
 
     def sample(self, text_c, text_u, height: int, width: int, steps: int = 50, cfg: float = 3.0, shift: float = 5.0,

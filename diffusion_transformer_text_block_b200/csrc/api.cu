@@ -203,6 +203,10 @@ struct moss_model {
   float* sc = nullptr;   // [max_steps, C]
   float* tvals = nullptr;
   int64_t mod_stride = 0;
+  // The schedule whose per-step modulation m->mod holds (rows 0..steps-1), or steps 0 when it
+  // holds something else (one timestep of a forward or block call).
+  int mod_sched_steps = 0;
+  double mod_sched_shift = 0.0;
   int rope_gh = -1, rope_gw = -1, rope_nt = -1;
   int rope_n = 0;  // tokens of the cached RoPE table (its pair-row stride)
   unsigned* err = nullptr;
@@ -212,6 +216,9 @@ struct moss_model {
   float* cache_res = nullptr;
   double* chg_dev = nullptr;
   double* chg_host = nullptr;  // pinned
+  // staging of moss_denoise_step_host (allocated on first use): the latent and both prompts
+  float* stage_x = nullptr;     // [max_latent_hw * 32]
+  float* stage_text = nullptr;  // [2 * max_tokens * D]
   // text path (moss_text_refiner_set): weights, descriptors, the blocks' fixed modulation
   bool has_text = false;
   moss_text_weights tw;
@@ -346,6 +353,7 @@ int ensure_rope(moss_model* m, int gh, int gw, int nt, cudaStream_t s) {
 int compute_modulation(moss_model* m, const float* ts_host, int T, cudaStream_t s) {
   const moss_config& c = m->cfg;
   const int D = c.hidden, L = c.layers, C = c.cond_dim;
+  m->mod_sched_steps = 0;  // the callers that hold a whole schedule record it afterwards
   MOSS_CUDA(cudaMemcpyAsync(m->tvals, ts_host, sizeof(float) * T, cudaMemcpyHostToDevice, s), "copy timesteps");
   LAUNCH(m, MOSS_K_OTHER, s,
          launch_conditioning(static_cast<const bf16*>(m->w.t_w1), static_cast<const bf16*>(m->w.t_b1),
@@ -360,6 +368,18 @@ int compute_modulation(moss_model* m, const float* ts_host, int T, cudaStream_t 
          launch_mod_gemv(static_cast<const bf16*>(m->w.final_mod_w), static_cast<const bf16*>(m->w.final_mod_b),
                          m->sc, m->mod + static_cast<int64_t>(L) * 6 * D, 2 * D, C, T, m->mod_stride, s),
          "final modulation");
+  return MOSS_OK;
+}
+
+// Modulation of every step of the (steps, shift) schedule sig in m->mod, computed unless m->mod
+// already holds exactly that schedule.  Requires steps <= max_steps.
+int ensure_schedule_modulation(moss_model* m, const std::vector<float>& sig, int steps, double shift,
+                               cudaStream_t s) {
+  if (m->mod_sched_steps == steps && m->mod_sched_shift == shift) return MOSS_OK;
+  const int rc = compute_modulation(m, sig.data(), steps, s);
+  if (rc) return rc;
+  m->mod_sched_steps = steps;
+  m->mod_sched_shift = shift;
   return MOSS_OK;
 }
 
@@ -811,8 +831,9 @@ int moss_model_create(const moss_config* cfg, const moss_weights* w, moss_model*
 void moss_model_free(moss_model* m) {
   if (!m) return;
   cudaDeviceSynchronize();
-  void* bufs[] = {m->x,   m->h,  m->qkv,   m->attn,      m->act,      m->patches, m->v,
-                  m->rope, m->mod, m->sc, m->tvals, m->cache_ref, m->cache_res, m->chg_dev, m->tt_mod};
+  void* bufs[] = {m->x,   m->h,  m->qkv,   m->attn,      m->act,      m->patches, m->v,       m->rope,
+                  m->mod, m->sc, m->tvals, m->cache_ref, m->cache_res, m->chg_dev, m->tt_mod, m->stage_x,
+                  m->stage_text};
   for (void* p : bufs)
     if (p) cudaFree(p);
   if (m->chg_host) cudaFreeHost(m->chg_host);
@@ -918,6 +939,26 @@ static int check_step_args(moss_model* m, float* x, const float* text_c, int n_t
   return MOSS_OK;
 }
 
+// The denoising step after its arguments have been checked (uskip: the parsed skip set).
+static int denoise_step_impl(moss_model* m, float* x, const float* text_c, int n_txt_c, const float* text_u,
+                             int n_txt_u, int height, int width, int step, int steps, float cfg, double shift,
+                             std::vector<char> uskip, double slg_start, double slg_stop, cudaStream_t s) {
+  int rc = MOSS_OK;
+  if (!slg_on(step, steps, slg_start, slg_stop)) std::fill(uskip.begin(), uskip.end(), 0);
+  std::vector<float> sig;
+  host_schedule(steps, shift, &sig);
+  const float* mod = m->mod;
+  if (steps <= m->cfg.max_steps) {
+    rc = ensure_schedule_modulation(m, sig, steps, shift, s);
+    mod = m->mod + static_cast<int64_t>(step) * m->mod_stride;
+  } else {
+    rc = compute_modulation(m, &sig[step], 1, s);
+  }
+  if (rc) return rc;
+  return step_impl(m, x, text_c, n_txt_c, text_u, n_txt_u, height, width, sig[step], sig[step + 1], cfg, uskip,
+                   mod, s);
+}
+
 int moss_denoise_step(moss_model* m, float* x, const float* text_c, int n_txt_c, const float* text_u, int n_txt_u,
                       int height, int width, int step, int steps, float cfg, double shift,
                       const int* uncond_skip_layers, int n_skip, double slg_start, double slg_stop, void* stream) {
@@ -925,17 +966,61 @@ int moss_denoise_step(moss_model* m, float* x, const float* text_c, int n_txt_c,
   if (steps < 1 || step < 0 || step >= steps || !(shift > 0.0))
     return fail(MOSS_ERR_INVALID_ARGUMENT, "need 0 <= step < steps and shift > 0");
   std::vector<char> uskip;
-  int rc = check_step_args(m, x, text_c, n_txt_c, text_u, n_txt_u, height, width, cfg, uncond_skip_layers, n_skip,
-                           &uskip);
+  const int rc = check_step_args(m, x, text_c, n_txt_c, text_u, n_txt_u, height, width, cfg, uncond_skip_layers,
+                                 n_skip, &uskip);
   if (rc) return rc;
-  if (!slg_on(step, steps, slg_start, slg_stop)) std::fill(uskip.begin(), uskip.end(), 0);
-  std::vector<float> sig;
-  host_schedule(steps, shift, &sig);
+  return denoise_step_impl(m, x, text_c, n_txt_c, text_u, n_txt_u, height, width, step, steps, cfg, shift, uskip,
+                           slg_start, slg_stop, static_cast<cudaStream_t>(stream));
+}
+
+int moss_denoise_step_host(moss_model* m, float* x_host, const float* text_c_host, int n_txt_c,
+                           const float* text_u_host, int n_txt_u, int height, int width, int step, int steps, float cfg,
+                           double shift, const int* uncond_skip_layers, int n_skip, double slg_start, double slg_stop,
+                           void* stream) {
+  g_last_error.clear();
+  if (steps < 1 || step < 0 || step >= steps || !(shift > 0.0))
+    return fail(MOSS_ERR_INVALID_ARGUMENT, "need 0 <= step < steps and shift > 0");
+  if (!m) return fail(MOSS_ERR_INVALID_ARGUMENT, "model is NULL");
+  if (!x_host || (n_txt_c > 0 && !text_c_host) || (cfg != 1.0f && n_txt_u > 0 && !text_u_host))
+    return fail(MOSS_ERR_INVALID_ARGUMENT, "x and text states must not be NULL");
+  if (n_txt_c < 0 || n_txt_u < 0) return fail(MOSS_ERR_INVALID_ARGUMENT, "text lengths must be >= 0");
+  int rc = check_size(height, width);
+  if (rc) return rc;
+  const bool two = cfg != 1.0f;
+  rc = check_tokens(m, two ? 2 : 1, height / 16, width / 16, two ? std::max(n_txt_c, n_txt_u) : n_txt_c);
+  if (rc) return rc;
+  std::vector<std::vector<char>> sk;
+  rc = parse_skips(m, 1, uncond_skip_layers, n_skip, &sk);
+  if (rc) return rc;
+  const int D = m->cfg.hidden;
+  if (!m->stage_x) {
+    const size_t bx = sizeof(float) * static_cast<size_t>(m->cfg.max_latent_hw) * 32;
+    const size_t bt = sizeof(float) * 2 * static_cast<size_t>(m->cfg.max_tokens) * D;
+    if (cudaMalloc(&m->stage_x, bx) != cudaSuccess || cudaMalloc(&m->stage_text, bt) != cudaSuccess) {
+      cudaGetLastError();
+      if (m->stage_x) cudaFree(m->stage_x);
+      m->stage_x = nullptr;
+      m->stage_text = nullptr;
+      return fail(MOSS_ERR_OOM, "cannot allocate the host-step staging buffers");
+    }
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  rc = compute_modulation(m, &sig[step], 1, s);
+  const size_t nx = static_cast<size_t>(height / 8) * (width / 8) * 32;
+  float* tc = m->stage_text;
+  float* tu = m->stage_text + static_cast<size_t>(m->cfg.max_tokens) * D;
+  MOSS_CUDA(cudaMemcpyAsync(m->stage_x, x_host, sizeof(float) * nx, cudaMemcpyHostToDevice, s), "copy latent in");
+  if (n_txt_c > 0)
+    MOSS_CUDA(cudaMemcpyAsync(tc, text_c_host, sizeof(float) * n_txt_c * D, cudaMemcpyHostToDevice, s),
+              "copy prompt in");
+  if (two && n_txt_u > 0)
+    MOSS_CUDA(cudaMemcpyAsync(tu, text_u_host, sizeof(float) * n_txt_u * D, cudaMemcpyHostToDevice, s),
+              "copy negative prompt in");
+  rc = denoise_step_impl(m, m->stage_x, tc, n_txt_c, tu, two ? n_txt_u : 0, height, width, step, steps, cfg, shift,
+                         sk[0], slg_start, slg_stop, s);
   if (rc) return rc;
-  return step_impl(m, x, text_c, n_txt_c, text_u, n_txt_u, height, width, sig[step], sig[step + 1], cfg, uskip,
-                   m->mod, s);
+  MOSS_CUDA(cudaMemcpyAsync(x_host, m->stage_x, sizeof(float) * nx, cudaMemcpyDeviceToHost, s), "copy latent out");
+  MOSS_CUDA(cudaStreamSynchronize(s), "host step");
+  return MOSS_OK;
 }
 
 int moss_sample(moss_model* m, int steps, float cfg, double shift, uint64_t seed, const int* uncond_skip_layers,
@@ -954,7 +1039,7 @@ int moss_sample(moss_model* m, int steps, float cfg, double shift, uint64_t seed
   LAUNCH(m, MOSS_K_OTHER, s, launch_noise(latent_out, n, seed, s), "noise");
   std::vector<float> sig;
   host_schedule(steps, shift, &sig);
-  rc = compute_modulation(m, sig.data(), steps, s);
+  rc = ensure_schedule_modulation(m, sig, steps, shift, s);
   if (rc) return rc;
   const std::vector<char> none(m->cfg.layers, 0);
   for (int i = 0; i < steps; ++i) {
@@ -1098,7 +1183,7 @@ int moss_sample_ex(moss_model* m, int steps, float cfg, double shift, uint64_t s
   LAUNCH(m, MOSS_K_OTHER, s, launch_noise(latent_out, n, seed, s), "noise");
   std::vector<float> sig;
   host_schedule(steps, shift, &sig);
-  rc = compute_modulation(m, sig.data(), steps, s);
+  rc = ensure_schedule_modulation(m, sig, steps, shift, s);
   if (rc) return rc;
   const std::vector<char> none(m->cfg.layers, 0);
   StepCache sc;

@@ -179,13 +179,14 @@ __global__ void noise_kernel(float* __restrict__ x, int64_t n, uint32_t k0, uint
 // ---------------------------------------------------------------------------- conditioning
 // c = W2 SiLU(W1 e + b1) + b2 with e = [cos, sin](1000 t exp(-ln(1e4) k / 128)); out SiLU(c),
 // the input of every modulation linear (InvokeAI MOSS-Image guide, Transformer formats: the
-// time-embedding and modulation layers).  One block per timestep, one thread per output.
-__global__ void cond_kernel(const bf16* __restrict__ w1, const bf16* __restrict__ b1, const bf16* __restrict__ w2,
-                            const bf16* __restrict__ b2, const float* __restrict__ ts, float* __restrict__ sc,
-                            int cdim) {
-  extern __shared__ float sm[];
-  float* emb = sm;          // [256]
-  float* hid = sm + 256;    // [cdim]
+// time-embedding and modulation layers).  One block per timestep; one warp per output row, its
+// lanes reading consecutive pieces of the row (one 16-byte load per lane for the 256-wide first
+// layer) and adding up with shuffles.
+__global__ void __launch_bounds__(256) cond_kernel(const bf16* __restrict__ w1, const bf16* __restrict__ b1,
+                                                   const bf16* __restrict__ w2, const bf16* __restrict__ b2,
+                                                   const float* __restrict__ ts, float* __restrict__ sc, int cdim) {
+  __shared__ float emb[256];
+  __shared__ float hid[256];
   const float t = ts[blockIdx.x];
   for (int k = threadIdx.x; k < 128; k += blockDim.x) {
     const double f = exp(-log(10000.0) * k / 128.0);
@@ -196,16 +197,34 @@ __global__ void cond_kernel(const bf16* __restrict__ w1, const bf16* __restrict_
     emb[128 + k] = static_cast<float>(s);
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < cdim; j += blockDim.x) {
-    float a = __bfloat162float(b1[j]);
-    for (int k = 0; k < 256; ++k) a = fmaf(__bfloat162float(w1[j * 256 + k]), emb[k], a);
-    hid[j] = a / (1.0f + expf(-a));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int j = warp; j < cdim; j += nwarps) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(w1 + static_cast<int64_t>(j) * 256) + lane);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(p[i]);
+      a = fmaf(f.x, emb[lane * 8 + 2 * i], a);
+      a = fmaf(f.y, emb[lane * 8 + 2 * i + 1], a);
+    }
+    a = warp_sum(a);
+    if (lane == 0) {
+      a += __bfloat162float(b1[j]);
+      hid[j] = a / (1.0f + expf(-a));
+    }
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < cdim; j += blockDim.x) {
-    float a = __bfloat162float(b2[j]);
-    for (int k = 0; k < cdim; ++k) a = fmaf(__bfloat162float(w2[j * cdim + k]), hid[k], a);
-    sc[static_cast<int64_t>(blockIdx.x) * cdim + j] = a / (1.0f + expf(-a));
+  const int per_lane = cdim / 32;  // cdim is a multiple of 32, at most 256
+  for (int j = warp; j < cdim; j += nwarps) {
+    const bf16* wr = w2 + static_cast<int64_t>(j) * cdim + lane * per_lane;
+    float a = 0.f;
+    for (int i = 0; i < per_lane; ++i) a = fmaf(__bfloat162float(wr[i]), hid[lane * per_lane + i], a);
+    a = warp_sum(a);
+    if (lane == 0) {
+      a += __bfloat162float(b2[j]);
+      sc[static_cast<int64_t>(blockIdx.x) * cdim + j] = a / (1.0f + expf(-a));
+    }
   }
 }
 
@@ -369,7 +388,7 @@ cudaError_t launch_noise(float* x, int64_t n, uint64_t seed, cudaStream_t s) {
 cudaError_t launch_conditioning(const bf16* w1, const bf16* b1, const bf16* w2, const bf16* b2, const float* ts,
                                 float* sc, int T, int cdim, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  cond_kernel<<<T, 256, (256 + cdim) * sizeof(float), s>>>(w1, b1, w2, b2, ts, sc, cdim);
+  cond_kernel<<<T, 256, 0, s>>>(w1, b1, w2, b2, ts, sc, cdim);
   return cudaGetLastError();
 }
 

@@ -199,10 +199,29 @@ int moss_init_noise(float* x, int64_t n, uint64_t seed, void* stream);
  *   x: device FP32 [height/8, width/8, 32]
  *   text_c: device FP32 [n_txt_c, D];  text_u: device FP32 [n_txt_u, D] (unused when cfg == 1)
  *   uncond_skip_layers: host int [n_skip] in 0..L-1.
+ * Modulation: when steps <= max_steps, the first call for a (steps, shift) schedule computes the
+ * modulation vectors of all its steps at once (one pass over the modulation weights, as
+ * moss_sample does) and later calls for the same schedule reuse them; a call of
+ * moss_dit_forward, moss_dit_block_forward or moss_op_modulation in between drops them.  With
+ * steps > max_steps each call computes its own step's vectors.  The weights are read-only for
+ * the model's lifetime, so the reused vectors always match them.
  * Errors: as moss_dit_forward; each branch's image + text tokens must fit max_tokens. */
 int moss_denoise_step(moss_model* m, float* x, const float* text_c, int n_txt_c, const float* text_u, int n_txt_u,
                       int height, int width, int step, int steps, float cfg, double shift,
                       const int* uncond_skip_layers, int n_skip, double slg_start, double slg_stop, void* stream);
+
+/* moss_denoise_step with host buffers: the same step, with x_host (host FP32 [height/8, width/8,
+ * 32], updated in place), text_c_host (host FP32 [n_txt_c, D]) and text_u_host (host FP32
+ * [n_txt_u, D], unused when cfg == 1) in host memory.  The call copies the latent and the prompts
+ * to the device on `stream`, runs the step there, copies the latent back and waits for the stream,
+ * so x_host holds the result when it returns.  Pinned (page-locked) host buffers make the copies
+ * asynchronous with the host; pageable ones work too, more slowly.  The device staging buffers
+ * (the latent and two prompts at the model's maxima) are allocated on the first call and kept until
+ * moss_model_free.  Errors: as moss_denoise_step; OOM if the staging buffers cannot be allocated. */
+int moss_denoise_step_host(moss_model* m, float* x_host, const float* text_c_host, int n_txt_c,
+                           const float* text_u_host, int n_txt_u, int height, int width, int step, int steps, float cfg,
+                           double shift, const int* uncond_skip_layers, int n_skip, double slg_start, double slg_stop,
+                           void* stream);
 
 /* The full sampling loop ([SGL-MOSS] 3 defaults: 50 steps, shift 5, CFG 3, empty negative,
  * uncond layer 22 skipped in slg 0.01..1.0): noise from `seed`, then `steps` calls of the

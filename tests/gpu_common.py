@@ -40,3 +40,26 @@ def psnr(ref, test) -> float:
     mse = float(np.mean((ref - test) ** 2))
     rng = float(ref.max() - ref.min())
     return float("inf") if mse == 0 else 10 * math.log10(rng * rng / mse)
+
+
+class LazyLayers:
+    """A stacked [L, ...] weight tensor on the GPU that the oracle indexes one layer at a time: each
+    index returns that layer as an exact float64 numpy copy.  The full model's 5e9 parameters in
+    float64 would need 40 GB of host memory; one layer needs under 1 GB."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __len__(self):
+        return self.shape[0]
+
+    def __getitem__(self, l):
+        return self.t[l].to(torch.float64).cpu().numpy()
+
+
+def lazy_numpy_weights(w: dict) -> dict:
+    """The oracle's view of a GPU weight dict: stacked per-layer weights stay on the GPU behind
+    LazyLayers, the small ones are copied to float64 numpy once."""
+    per_layer = {"mod_w", "mod_b", "wqkv", "q_gain", "k_gain", "wo", "wg", "wu", "wd"}
+    return {k: LazyLayers(v) if k in per_layer else to_numpy(v) for k, v in w.items()}
