@@ -283,6 +283,56 @@ def run_op(args):
     return 0
 
 
+def run_cfg_euler(args):
+    """The standalone CFG + Euler kernel (moss_cfg_euler_step) on the 1024^2 and 2048^2 latents
+    (128x128x32 and 256x256x32 FP32): x, v_c and v_u only.  Each launch takes the next of enough
+    buffer sets that together exceed L2 twice over, so every launch streams from HBM.  Prints one JSON
+    line: per size the mean device time per launch and the algorithmic HBM bytes (read x, v_c, v_u;
+    write x: 16 B per element) over that time.  The launches are captured once in a CUDA graph and
+    the graph is replayed between CUDA events, so the host's per-call cost (about 12 us through the
+    Python binding, longer than the kernel itself) does not pace the device."""
+    import torch
+
+    import diffusion_transformer_text_block_b200 as moss
+
+    peaks = read_peaks()
+    out = {"op": "cfg_euler", "l2": "buffer sets rotated, 2 x L2 in total", "sizes": {}}
+    for side in (1024, 2048):
+        n = (side // 8) * (side // 8) * 32
+        sets = max(2, int(2 * 126e6 // (12 * n)) + 1)
+        bufs = [[torch.randn(n, device="cuda") for _ in range(3)] for _ in range(sets)]
+        for i in range(max(args.warmup, 3)):
+            x, c, u = bufs[i % sets]
+            moss.cfg_euler_step(x, c, u, 3.0, 0.9, 0.8)
+        torch.cuda.synchronize()
+        launches = max(args.steps, 2 * sets)
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(graph, stream=cap):
+                for i in range(launches):
+                    x, c, u = bufs[i % sets]
+                    moss.cfg_euler_step(x, c, u, 3.0, 0.9, 0.8)
+        graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / launches
+        del graph
+        gbs = 16.0 * n / (us * 1e-6) / 1e9
+        out["sizes"][f"{side}^2"] = {"elements": n, "bytes_per_launch": 16 * n, "us_per_launch": round(us, 3),
+                                     "gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+                                     "launches": launches, "buffer_sets": sets}
+        del bufs
+    out["peak_source"] = f"{peaks['source']} hbm {peaks['hbm_gbs']} GB/s"
+    out["device_status"] = moss.device_status(clear=True)
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def run_c5(args):
     """The long-sequence stress workload: 2048^2 (16384 image tokens) with a 4096-token prompt
     (20480 tokens per branch), full 42-block DiT, CFG batch 2, skip layer 22, 10 Euler steps at
@@ -438,7 +488,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["block", "attention", "accel", "text", "c5"], default=None,
+    ap.add_argument("--op", choices=["block", "attention", "accel", "text", "c5", "cfg_euler"], default=None,
                     help="time one kernel class on the 1024^2 shapes instead of the denoising step; "
                          "'accel' times whole 50-step images with the lossy accelerators")
     args = ap.parse_args()
@@ -450,6 +500,8 @@ def main():
         return run_text(args)
     if args.op == "c5":
         return run_c5(args)
+    if args.op == "cfg_euler":
+        return run_cfg_euler(args)
     if args.op:
         return run_op(args)
 
@@ -606,7 +658,9 @@ def main():
         "tc_frac_step": round(tc_frac, 4),
         "roofline": roofline, "kernels": kernels,
         "kernels_note": f"per-class device time from a profiled pass of {prof_steps} steps after the timed region "
-                        "(the timed region itself times only the gemm_gateup and attention launches)",
+                        "(the timed region itself times only the gemm_gateup and attention launches); the CFG + "
+                        "Euler update runs inside the output projection (class 'other'), so 'cfg_euler' has no "
+                        "launches in the step; bench.py --op cfg_euler times the standalone kernel",
         "cpu_baseline": cb, "e2e": e2e,
         "clocks": clocks.summary(), "gpu_launches": launches, "device_status": status,
     }

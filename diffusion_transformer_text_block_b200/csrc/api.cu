@@ -563,6 +563,29 @@ int final_impl(moss_model* m, const CallRows& r, const float* mod, float* v_out,
   return MOSS_OK;
 }
 
+// Final layer of a guided two-branch step fused with its update: LN-modulate of both branches'
+// image rows, then one kernel that projects the conditional and the unconditional rows of each
+// token tile and applies x += (sigma_next - sigma) (v_u + cfg (v_c - v_u)) to the latent in FP32.
+int final_cfg_impl(moss_model* m, const CallRows& r, const float* mod, float* x, float cfg, float sigma,
+                   float sigma_next, cudaStream_t s) {
+  const int D = m->cfg.hidden, L = m->cfg.layers;
+  const float* fmod = mod + static_cast<int64_t>(L) * 6 * D;
+  const int rows = 2 * r.n_img;
+  LAUNCH(m, MOSS_K_LN_MOD, s, launch_ln_mod(m->x, fmod, fmod + D, m->h, rows, D, r.n_img, r.lens[0], 1e-6f, s),
+         "final ln");
+  std::string e;
+  CUtensorMap tm_hf;
+  if (!make_tmap_bf16_2d(&tm_hf, m->h, D, rows, kGemmBoxK, kGemmBoxRows, &e)) return fail(MOSS_ERR_CUDA, e);
+  EpiParams oe;
+  oe.M = rows; oe.N = 128; oe.K = D;
+  oe.bias = static_cast<const bf16*>(m->w.out_b);
+  oe.n_img = r.n_img; oe.grid_w = r.gw; oe.lat_h8 = r.h8; oe.lat_w8 = r.w8;
+  oe.x_lat = x; oe.cfg = cfg; oe.dt = sigma_next - sigma;
+  LAUNCH(m, MOSS_K_OTHER, s, launch_gemm(kEpiOutCfg, tm_hf, m->tm_out, m->tm_out, oe, s, m->err),
+         "output projection with cfg euler");
+  return MOSS_OK;
+}
+
 int forward_impl(moss_model* m, int batch, const float* latent, const float* const* texts, const int* n_txts,
                  int height, int width, const float* mod, const std::vector<std::vector<char>>& skip, float* v_out,
                  cudaStream_t s) {
@@ -596,6 +619,13 @@ int step_impl(moss_model* m, float* x, const float* text_c, int n_txt_c, const f
   if (batch == 2) skips[1] = uskip;
   const float* texts[2] = {text_c, text_u};
   const int n_txts[2] = {n_txt_c, n_txt_u};
+  if (batch == 2) {  // the guided step: the update is part of the output projection
+    CallRows r;
+    int rc = embed_impl(m, batch, x, texts, n_txts, height, width, &r, s);
+    if (!rc) rc = blocks_impl(m, 0, m->cfg.layers, r, mod, skips, s);
+    if (!rc) rc = final_cfg_impl(m, r, mod, x, cfg, sigma, sigma_next, s);
+    return rc;
+  }
   int rc = forward_impl(m, batch, x, texts, n_txts, height, width, mod, skips, m->v, s);
   if (rc) return rc;
   const int64_t n = static_cast<int64_t>(height / 8) * (width / 8) * 32;

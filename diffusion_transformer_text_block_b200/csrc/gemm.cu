@@ -22,7 +22,12 @@
 // of two independent 128-row CTAs, and a 32 KB slot allows a six-deep ring.
 // Tiles are visited in bands of 16 M-tiles (all N-tiles of a band before the next band).
 //
-// The 128 x 128 output projection (`gemm_kernel`, BN = 128) keeps the single-CTA form.
+// The 128 x 128 output projection (`gemm_kernel`, BN = 128) keeps the single-CTA form.  In the
+// guided step its CFG form (kEpiOutCfg) gives each CTA one tile of 128 image tokens: the MMA warp
+// accumulates the conditional rows into the first accumulator and the unconditional rows of the
+// same tokens into the second, and the epilogue applies the FP32 CFG combine and Euler update to
+// the latent directly (SGLang cookbook, MOSS-Image: 3. Guidance and precision), so the step needs
+// no separate update kernel and no velocity round trip through memory.
 //
 // Epilogues follow the block of the single-stream DiT (windpaint.ai, MOSS-Image specs:
 // 24 heads of 128, FFN 8192) with the fused tails the sibling DiT names on B200 (SGLang
@@ -303,6 +308,43 @@ __device__ __forceinline__ void epi_out(const EpiParams& ep, uint32_t tb, int ro
   }
 }
 
+// Token tile u of the guided step: accumulator 0 = conditional rows, accumulator 1 = the
+// unconditional rows of the same tokens (tb1 = tb0 + 128).  x[lat] += dt * (v_u + cfg (v_c - v_u))
+// with v = acc + bias, in the order and rounding of the standalone CFG + Euler kernel.
+__device__ __forceinline__ void epi_out_cfg(const EpiParams& ep, uint32_t tb0, int tok, int half) {
+  const bool valid = tok < ep.n_img;
+  const int r = tok / ep.grid_w;
+  const int cc = tok - r * ep.grid_w;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int c = half * 2 + q;
+    float vc[32], vu[32];
+    tmem_ld32f(tb0 + c * 32, vc);
+    tmem_ld32f(tb0 + 128 + c * 32, vu);
+    if (valid) {
+      const int dy = c >> 1, dx = c & 1;
+      float4* xp = reinterpret_cast<float4*>(
+          ep.x_lat + ((static_cast<int64_t>(2 * r + dy) * ep.lat_w8) + 2 * cc + dx) * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 a = xp[i];
+        float cv[4], uv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float bj = __bfloat162float(ep.bias[c * 32 + 4 * i + e]);
+          cv[e] = vc[4 * i + e] + bj;
+          uv[e] = vu[4 * i + e] + bj;
+        }
+        a.x = fmaf(ep.dt, fmaf(ep.cfg, cv[0] - uv[0], uv[0]), a.x);
+        a.y = fmaf(ep.dt, fmaf(ep.cfg, cv[1] - uv[1], uv[1]), a.y);
+        a.z = fmaf(ep.dt, fmaf(ep.cfg, cv[2] - uv[2], uv[2]), a.z);
+        a.w = fmaf(ep.dt, fmaf(ep.cfg, cv[3] - uv[3], uv[3]), a.w);
+        xp[i] = a;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------------ the kernel
 // Ten warps: three share one SM sub-partition, whose register file caps them at 168 each.
 template <int BN, int EPI>
@@ -324,9 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // kEpiOutCfg: a work unit is one tile of 128 image tokens made of two consecutive tiles, the
+  // conditional rows (accumulator 0) and the unconditional rows (accumulator 1); otherwise a unit
+  // is one output tile.
+  constexpr int kPer = EPI == kEpiOutCfg ? 2 : 1;
   const int num_m = (ep.M + kBM - 1) / kBM;
   const int num_n = (ep.N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
+  const int num_units = EPI == kEpiOutCfg ? (ep.n_img + kBM - 1) / kBM : num_m * num_n;
   const int num_kb = ep.K / kBK;
 
   if (threadIdx.x == 0) {
@@ -363,24 +409,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       int armed[S::kStages];  // parity of the last phase armed on full[s], -1 = never
 #pragma unroll
       for (int s2 = 0; s2 < S::kStages; ++s2) armed[s2] = -1;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, num_m, num_n, mb, nb);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, err, kErrGemmProducer, abort_flag)) {
-            ok = false;
-            break;
+      for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x)
+        for (int sub = 0; sub < kPer && ok; ++sub) {
+          int arow, brow;
+          if constexpr (EPI == kEpiOutCfg) {
+            arow = sub * ep.n_img + unit * kBM;  // branch `sub`, tokens unit*128 ..
+            brow = 0;
+          } else {
+            int mb, nb;
+            tile_coords(unit, num_m, num_n, mb, nb);
+            arow = mb * kBM;
+            brow = nb * BN;
           }
-          armed[stage] = static_cast<int>(phase);
-          mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
-          tma_load_2d(sA + stage * S::kABytes, &tmA, &full[stage], kb * kBK, mb * kBM);
-          tma_load_2d(sB + stage * S::kBBytes, &tmB, &full[stage], kb * kBK, nb * BN);
-          if (++stage == S::kStages) {
-            stage = 0;
-            phase ^= 1;
+          for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, err, kErrGemmProducer, abort_flag)) {
+              ok = false;
+              break;
+            }
+            armed[stage] = static_cast<int>(phase);
+            mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+            tma_load_2d(sA + stage * S::kABytes, &tmA, &full[stage], kb * kBK, arow);
+            tma_load_2d(sB + stage * S::kBBytes, &tmB, &full[stage], kb * kBK, brow);
+            if (++stage == S::kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
         }
-      }
       if (!ok) {
         // Let the loads already issued land before the CTA can exit (bounded as well).
         for (int s2 = 0; s2 < S::kStages; ++s2) {
@@ -399,7 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      const int num_tiles = num_units * kPer;  // this CTA's tiles come in runs of kPer (one unit)
+      for (int tile = blockIdx.x * kPer; tile < num_tiles && ok;
+           tile += (tile % kPer == kPer - 1) ? (gridDim.x - 1) * kPer + 1 : 1, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, err, kErrGemmMma, abort_flag)) break;
@@ -439,7 +496,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;          // TMEM lane quadrant this warp may access
     const int half = (warp - 2) >> 2;   // which half of the tile's columns it owns
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    if constexpr (EPI == kEpiOutCfg) {
+      // Both accumulators of a unit (it even: accumulator 0, then 1 in the same phase).
+      for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, it += 2) {
+        const uint32_t acc_phase = (it >> 1) & 1;
+        const bool ok = mbar_wait(&tfull[0], acc_phase, err, kErrGemmEpilogue, abort_flag) &&
+                        mbar_wait(&tfull[1], acc_phase, err, kErrGemmEpilogue, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: TMEM loads are .sync.aligned
+        tc_fence_after();
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+        epi_out_cfg(ep, tb, unit * kBM + quad * 32 + lane, half);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&tempty[0]);
+          mbar_arrive(&tempty[1]);
+        }
+      }
+    }
+    for (int tile = blockIdx.x; EPI != kEpiOutCfg && tile < num_units; tile += gridDim.x, ++it) {
       int mb, nb;
       tile_coords(tile, num_m, num_n, mb, nb);
       const int acc = it & 1;
@@ -678,7 +753,8 @@ cudaError_t launch_single(const CUtensorMap& a, const CUtensorMap& b, const EpiP
     if (e != cudaSuccess) return e;
     mark_configured_on_device(configured);
   }
-  const int tiles = ((ep.M + kBM - 1) / kBM) * ((ep.N + BN - 1) / BN);
+  const int tiles = EPI == kEpiOutCfg ? (ep.n_img + kBM - 1) / kBM
+                                     : ((ep.M + kBM - 1) / kBM) * ((ep.N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (grid <= 0) return cudaSuccess;
   gemm_kernel<BN, EPI><<<grid, kThreads, S::kSmemBytes, s>>>(a, b, b, ep, err);
@@ -723,6 +799,7 @@ cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& a, const CUtensorMap& b
     case kEpiSwiglu: return launch_pair<kEpiSwiglu>(a, b, b2, ep, s, err);
     case kEpiEmbed: return launch_pair<kEpiEmbed>(a, b, b2, ep, s, err);
     case kEpiOut: return launch_single<128, kEpiOut>(a, b, ep, s, err);
+    case kEpiOutCfg: return launch_single<128, kEpiOutCfg>(a, b, ep, s, err);
   }
   return cudaErrorInvalidValue;
 }

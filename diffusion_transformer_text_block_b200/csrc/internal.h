@@ -38,6 +38,7 @@ enum EpiKind : int {
   kEpiSwiglu = 3,  // act = BF16(SiLU(acc_gate) * acc_up)
   kEpiEmbed = 4,   // x[b, row, :] = acc + bias for every branch b
   kEpiOut = 5,     // unpatchified velocity = acc + bias
+  kEpiOutCfg = 6,  // both branches' velocities of one token tile, then the CFG + Euler update of x
 };
 
 struct EpiParams {
@@ -56,7 +57,9 @@ struct EpiParams {
                                      // branches of n_tok tokens (token = row % n_tok)
   int hidden = 0;                    // D
   int n_branch = 0;                  // kEpiEmbed: branches written
-  int n_img = 0, grid_w = 0, lat_h8 = 0, lat_w8 = 0;  // kEpiOut
+  int n_img = 0, grid_w = 0, lat_h8 = 0, lat_w8 = 0;  // kEpiOut, kEpiOutCfg
+  float* x_lat = nullptr;            // kEpiOutCfg: the latent [lat_h8, lat_w8, 32], updated in place
+  float cfg = 1.0f, dt = 0.0f;       // kEpiOutCfg: guidance scale, sigma_next - sigma
   float eps = 1e-6f;
 };
 

@@ -267,6 +267,38 @@ def test_full_denoise_step_matches_manual_cfg(full_model):
     assert_no_device_error()
 
 
+def test_full_guided_step_fused_update_matches_forward_and_update(full_model):
+    """The guided step applies the CFG + Euler update inside the output projection (one kernel per
+    tile of 128 image tokens, both branches).  On a 272^2 image (17 x 17 = 289 image tokens, so the
+    last token tile is partial) with a 300-token prompt and a 77-token negative prompt, it equals the
+    two branch forwards followed by the standalone CFG + Euler kernel, bit for bit."""
+    from synth import FULL
+    model, w = full_model
+    x0 = make_latent(34, 34, 24, device="cuda")
+    tc = make_text(1, 300, FULL.hidden, 25, device="cuda")[0].contiguous()
+    tu = make_text(1, 77, FULL.hidden, 26, device="cuda")[0].contiguous()
+    x = x0.clone()
+    before = moss.launch_count()
+    model.denoise_step(x, tc, tu, 272, 272, 7, 50, 3.0, 5.0, [22], 0.01, 1.0)
+    fused_launches = moss.launch_count() - before
+    sig = o.sigma_schedule(50, 5.0)
+    vc = model.forward(x0, tc[None], 272, 272, float(sig[7]), skip_layers=[[]]).clone()
+    vu = model.forward(x0, tu[None], 272, 272, float(sig[7]), skip_layers=[[22]]).clone()
+    ref = x0.clone()
+    moss.cfg_euler_step(ref, vc[0].contiguous(), vu[0].contiguous(), 3.0, float(sig[7]), float(sig[8]))
+    torch.cuda.synchronize()
+    assert torch.equal(x, ref)
+    assert rel_l2(x.cpu().numpy(), x0.cpu().numpy()) > 1e-3
+    # the step launched no standalone update kernel: its class saw no launch
+    model.profile_enable(True)
+    model.denoise_step(x, tc, tu, 272, 272, 8, 50, 3.0, 5.0, [22], 0.01, 1.0)
+    prof = model.profile_read()
+    model.profile_enable(False)
+    assert prof["cfg_euler"][0] == 0 and prof["gemm_qkv"][0] > 0
+    assert fused_launches > 0
+    assert_no_device_error()
+
+
 @pytest.mark.parametrize("n_u", [5, 0])
 def test_sample_tiny_short_negative_prompt(n_u):
     """Branches of different text lengths (n_u = 0: the empty negative prompt): the tiny
