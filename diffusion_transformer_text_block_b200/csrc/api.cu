@@ -398,6 +398,12 @@ struct LayerRes {
   const float* k_gain;
 };
 
+// M-tiles per band of the pair GEMMs' tile order, per GEMM of the block, chosen by DRAM bytes per
+// launch at the 1024^2 shape (M = 9216, 36 pair tiles along M) with equal launch times: down (K =
+// 8192) reads 639 MB with bands of 4 against 751 MB with 16 (its 4 MB activation band per M-tile
+// stays in L2 across the N-tiles), O-proj 199 against 218 MB with 8, QKV and gate/up least with 16.
+constexpr int kBandQkv = 16, kBandOproj = 8, kBandGateUp = 16, kBandDown = 4;
+
 int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<int>& lens, const float* mod_l,
                  cudaStream_t s) {
   const moss_config& c = m->cfg;
@@ -427,6 +433,7 @@ int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<
   // order them so), the last one starts at split_rows.
   q.split_rows = equal ? 0 : static_cast<int>(M - lens[nb - 1]);
   q.rope_stride = m->rope_n;
+  q.group_m = kBandQkv;
   LAUNCH(m, MOSS_K_GEMM_QKV, s, launch_gemm(kEpiQkv, tm_h, *lw.qkv, *lw.qkv, q, s, m->err), "qkv gemm");
 
   if (equal) {
@@ -445,6 +452,7 @@ int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<
   EpiParams o;
   o.M = M; o.N = D; o.K = D;
   o.out_f32 = x; o.gate = mod_l + 2 * D;
+  o.group_m = kBandOproj;
   LAUNCH(m, MOSS_K_GEMM_OPROJ, s, launch_gemm(kEpiResid, tm_attn, *lw.wo, *lw.wo, o, s, m->err),
          "out-projection gemm");
 
@@ -454,12 +462,14 @@ int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<
   EpiParams g;
   g.M = M; g.N = F; g.K = D;
   g.out_bf16 = m->act;
+  g.group_m = kBandGateUp;
   LAUNCH(m, MOSS_K_GEMM_GATEUP, s, launch_gemm(kEpiSwiglu, tm_h, *lw.wg, *lw.wu, g, s, m->err),
          "gate/up gemm");
 
   EpiParams d;
   d.M = M; d.N = D; d.K = F;
   d.out_f32 = x; d.gate = mod_l + 5 * D;
+  d.group_m = kBandDown;
   LAUNCH(m, MOSS_K_GEMM_DOWN, s, launch_gemm(kEpiResid, tm_act, *lw.wd, *lw.wd, d, s, m->err),
          "down gemm");
   return MOSS_OK;

@@ -20,7 +20,8 @@
 //               barrier.  RoPE angles are read before waiting for the accumulator.
 // Each CTA streams half of every B tile, so a pair moves 3/4 of the operand bytes per output
 // of two independent 128-row CTAs, and a 32 KB slot allows a six-deep ring.
-// Tiles are visited in bands of 16 M-tiles (all N-tiles of a band before the next band).
+// Tiles are visited in bands of group_m M-tiles (all N-tiles of a band before the next band; the
+// launch chooses group_m per GEMM shape, 16 by default).
 //
 // The 128 x 128 output projection (`gemm_kernel`, BN = 128) keeps the single-CTA form.  In the
 // guided step its CFG form (kEpiOutCfg) gives each CTA one tile of 128 image tokens: the MMA warp
@@ -76,11 +77,11 @@ struct PairShape {
   static_assert(kSmemBytes <= 227 * 1024, "pair GEMM shared memory");
 };
 
-__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
-  const int band = tile / (kGroupM * num_n);
-  const int m0 = band * kGroupM;
-  const int bm = min(kGroupM, num_m - m0);
-  const int idx = tile - band * kGroupM * num_n;
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb, int group_m = kGroupM) {
+  const int band = tile / (group_m * num_n);
+  const int m0 = band * group_m;
+  const int bm = min(group_m, num_m - m0);
+  const int idx = tile - band * group_m * num_n;
   mb = m0 + idx % bm;
   nb = idx / bm;
 }
@@ -578,6 +579,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int num_n = EPI == kEpiSwiglu ? (ep.N + 127) / 128 : (ep.N + kTileN - 1) / kTileN;
   const int num_tiles = num_m * num_n;
   const int num_kb = ep.K / kBK;
+  const int group_m = ep.group_m > 0 ? ep.group_m : kGroupM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
@@ -619,7 +621,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const CUtensorMap* bmap = (EPI == kEpiSwiglu && !leader) ? &tmB2 : &tmB;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         int mb, nb;
-        tile_coords(tile, num_m, num_n, mb, nb);
+        tile_coords(tile, num_m, num_n, mb, nb, group_m);
         // Even CTA: gate rows (SwiGLU) or B rows 0..127 of the tile; odd CTA: up rows or 128..255.
         const int brow = EPI == kEpiSwiglu ? nb * 128 : nb * kTileN + static_cast<int>(rank) * 128;
         const int arow = mb * kTileM + static_cast<int>(rank) * kBM;
@@ -703,7 +705,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
       int mb, nb;
-      tile_coords(tile, num_m, num_n, mb, nb);
+      tile_coords(tile, num_m, num_n, mb, nb, group_m);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       const int row0 = mb * kTileM + static_cast<int>(rank) * kBM + quad * 32;

@@ -61,6 +61,8 @@ struct EpiParams {
   float* x_lat = nullptr;            // kEpiOutCfg: the latent [lat_h8, lat_w8, 32], updated in place
   float cfg = 1.0f, dt = 0.0f;       // kEpiOutCfg: guidance scale, sigma_next - sigma
   float eps = 1e-6f;
+  int group_m = 16;                  // pair GEMMs: M-tiles per band of the tile order (all N-tiles of
+                                     // a band before the next band)
 };
 
 // ------------------------------------------------------------------ tensor maps
