@@ -228,6 +228,7 @@ struct moss_model {
   // weight descriptors
   std::vector<CUtensorMap> tm_qkv, tm_wo, tm_wg, tm_wu, tm_wd;
   CUtensorMap tm_img, tm_out;
+  CUtensorMap tm_out64;  // out_w with a box of 64 rows: the guided output projection's half-width tiles
   // profiling
   bool prof = false;
   unsigned prof_mask = 0xFFFFFFFFu;  // classes timed while prof is on
@@ -575,7 +576,8 @@ int final_impl(moss_model* m, const CallRows& r, const float* mod, float* v_out,
 
 // Final layer of a guided two-branch step fused with its update: LN-modulate of both branches'
 // image rows, then one kernel that projects the conditional and the unconditional rows of each
-// token tile and applies x += (sigma_next - sigma) (v_u + cfg (v_c - v_u)) to the latent in FP32.
+// token tile (per CTA: 128 tokens, 64 of the 128 patch features) and applies
+// x += (sigma_next - sigma) (v_u + cfg (v_c - v_u)) to the latent in FP32.
 int final_cfg_impl(moss_model* m, const CallRows& r, const float* mod, float* x, float cfg, float sigma,
                    float sigma_next, cudaStream_t s) {
   const int D = m->cfg.hidden, L = m->cfg.layers;
@@ -591,7 +593,7 @@ int final_cfg_impl(moss_model* m, const CallRows& r, const float* mod, float* x,
   oe.bias = static_cast<const bf16*>(m->w.out_b);
   oe.n_img = r.n_img; oe.grid_w = r.gw; oe.lat_h8 = r.h8; oe.lat_w8 = r.w8;
   oe.x_lat = x; oe.cfg = cfg; oe.dt = sigma_next - sigma;
-  LAUNCH(m, MOSS_K_OTHER, s, launch_gemm(kEpiOutCfg, tm_hf, m->tm_out, m->tm_out, oe, s, m->err),
+  LAUNCH(m, MOSS_K_OTHER, s, launch_gemm(kEpiOutCfg, tm_hf, m->tm_out64, m->tm_out64, oe, s, m->err),
          "output projection with cfg euler");
   return MOSS_OK;
 }
@@ -860,7 +862,8 @@ int moss_model_create(const moss_config* cfg, const moss_weights* w, moss_model*
                         &m->tm_wd, &e))
     return cleanup(MOSS_ERR_CUDA, e);
   if (!make_tmap_bf16_2d(&m->tm_img, w->img_w, 128, D, kGemmBoxK, kGemmBoxRows, &e) ||
-      !make_tmap_bf16_2d(&m->tm_out, w->out_w, D, 128, kGemmBoxK, kGemmBoxRows, &e))
+      !make_tmap_bf16_2d(&m->tm_out, w->out_w, D, 128, kGemmBoxK, kGemmBoxRows, &e) ||
+      !make_tmap_bf16_2d(&m->tm_out64, w->out_w, D, 128, kGemmBoxK, 64, &e))
     return cleanup(MOSS_ERR_CUDA, e);
   cudaError_t ce = cudaDeviceSynchronize();
   if (ce != cudaSuccess) return cleanup(MOSS_ERR_CUDA, std::string("model creation: ") + cudaGetErrorString(ce));

@@ -229,39 +229,57 @@ __global__ void __launch_bounds__(256) cond_kernel(const bf16* __restrict__ w1, 
 }
 
 // ---------------------------------------------------------------------------- modulation
-// out[t, r] = W[r, :] . sc[t, :] + bias[r].  One warp per weight row, read once for all T
-// timesteps; cdim = 256 gives one 16-byte load per lane.
+// out[t, r] = W[r, :] . sc[t, :] + bias[r], FP32 sums of BF16 weights and FP32 inputs.  One thread
+// per weight row, so that a warp's results for one timestep are 32 consecutive floats (one
+// coalesced store); the timesteps are taken TC at a time with FP32 accumulators in registers, the
+// row read in 16-byte pieces (again from L1/L2 for each further chunk of timesteps), the inputs
+// sc[t, :] broadcast from shared memory.
+template <int TC>
 __global__ void __launch_bounds__(256) mod_gemv_kernel(const bf16* __restrict__ W, const bf16* __restrict__ bias,
                                                        const float* __restrict__ sc, float* __restrict__ out, int R,
                                                        int cdim, int T, int64_t out_stride) {
   extern __shared__ float s_sc[];  // [T, cdim]
   for (int i = threadIdx.x; i < T * cdim; i += blockDim.x) s_sc[i] = sc[i];
   __syncthreads();
-  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= R) return;
-  const int per_lane = cdim / 32;  // 8 for cdim = 256
-  float w[8];
-  const bf16* wr = W + static_cast<int64_t>(r) * cdim + lane * per_lane;
-  if (per_lane == 8) {
-    const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(wr));
-    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(p[i]);
-      w[2 * i] = f.x;
-      w[2 * i + 1] = f.y;
-    }
-  } else {
-    for (int i = 0; i < per_lane; ++i) w[i] = __bfloat162float(wr[i]);
-  }
+  const uint4* wr = reinterpret_cast<const uint4*>(W + static_cast<int64_t>(r) * cdim);
   const float bv = __bfloat162float(bias[r]);
-  for (int t = 0; t < T; ++t) {
-    const float* s = s_sc + t * cdim + lane * per_lane;
-    float a = 0.f;
-    for (int i = 0; i < per_lane; ++i) a = fmaf(w[i], s[i], a);
-    a = warp_sum(a);
-    if (lane == 0) out[t * out_stride + r] = a + bv;
+  for (int t0 = 0; t0 < T; t0 += TC) {
+    float acc[TC];
+#pragma unroll
+    for (int tt = 0; tt < TC; ++tt) acc[tt] = 0.f;
+    for (int k8 = 0; k8 < cdim / 8; ++k8) {
+      const uint4 raw = __ldg(wr + k8);
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      float w[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(p[i]);
+        w[2 * i] = f.x;
+        w[2 * i + 1] = f.y;
+      }
+#pragma unroll
+      for (int tt = 0; tt < TC; ++tt) {
+        if (TC == 1 || t0 + tt < T) {
+          const float4* sp = reinterpret_cast<const float4*>(s_sc + (t0 + tt) * cdim + 8 * k8);
+          const float4 s0 = sp[0], s1 = sp[1];
+          float a = acc[tt];
+          a = fmaf(w[0], s0.x, a);
+          a = fmaf(w[1], s0.y, a);
+          a = fmaf(w[2], s0.z, a);
+          a = fmaf(w[3], s0.w, a);
+          a = fmaf(w[4], s1.x, a);
+          a = fmaf(w[5], s1.y, a);
+          a = fmaf(w[6], s1.z, a);
+          a = fmaf(w[7], s1.w, a);
+          acc[tt] = a;
+        }
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < TC; ++tt)
+      if (TC == 1 || t0 + tt < T) out[static_cast<int64_t>(t0 + tt) * out_stride + r] = acc[tt] + bv;
   }
 }
 
@@ -398,11 +416,17 @@ cudaError_t launch_mod_gemv(const bf16* W, const bf16* bias, const float* sc, fl
   const size_t smem = static_cast<size_t>(T) * cdim * sizeof(float);
   static std::atomic<uint64_t> configured{0};
   if (!configured_on_device(configured)) {
-    const cudaError_t e = cudaFuncSetAttribute(mod_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(mod_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(mod_gemv_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (e != cudaSuccess) return e;
     mark_configured_on_device(configured);
   }
-  mod_gemv_kernel<<<(R + 7) / 8, 256, smem, s>>>(W, bias, sc, out, R, cdim, T, out_stride);
+  const unsigned blocks = static_cast<unsigned>((R + 255) / 256);
+  if (T == 1)
+    mod_gemv_kernel<1><<<blocks, 256, smem, s>>>(W, bias, sc, out, R, cdim, T, out_stride);
+  else
+    mod_gemv_kernel<16><<<blocks, 256, smem, s>>>(W, bias, sc, out, R, cdim, T, out_stride);
   return cudaGetLastError();
 }
 

@@ -24,10 +24,10 @@
 // launch chooses group_m per GEMM shape, 16 by default).
 //
 // The 128 x 128 output projection (`gemm_kernel`, BN = 128) keeps the single-CTA form.  In the
-// guided step its CFG form (kEpiOutCfg) gives each CTA one tile of 128 image tokens: the MMA warp
-// accumulates the conditional rows into the first accumulator and the unconditional rows of the
-// same tokens into the second, and the epilogue applies the FP32 CFG combine and Euler update to
-// the latent directly (SGLang cookbook, MOSS-Image: 3. Guidance and precision), so the step needs
+// guided step its CFG form (kEpiOutCfg, 128 x 64 tiles) gives each CTA one tile of 128 image tokens
+// and one half of the 128 patch features: the MMA warp accumulates the conditional rows into the
+// first accumulator and the unconditional rows of the same tokens into the second, and the epilogue
+// applies the FP32 CFG combine and Euler update to the latent directly (SGLang cookbook, MOSS-Image: 3. Guidance and precision), so the step needs
 // no separate update kernel and no velocity round trip through memory.
 //
 // Epilogues follow the block of the single-stream DiT (windpaint.ai, MOSS-Image specs:
@@ -49,9 +49,11 @@ constexpr int kGroupM = 16;
 constexpr int kResidStageBytes = static_cast<int>(kResidBoxCols * kResidBoxRows * 4);  // 2 KB per buffer
 constexpr int kThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 
+// The B map of a single-CTA GEMM has a box of BN rows (kGemmBoxRows for BN = 128, 64 rows for the
+// guided output projection's half-width tiles), so that B is one box per slot.
 template <int BN>
 struct GemmShape {
-  static_assert(BN == static_cast<int>(kGemmBoxRows), "single-CTA tiles load B with one box");
+  static_assert(BN == static_cast<int>(kGemmBoxRows) || BN == 64, "single-CTA tiles load B with one box");
   static constexpr int kStages = 6;
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
@@ -309,39 +311,38 @@ __device__ __forceinline__ void epi_out(const EpiParams& ep, uint32_t tb, int ro
   }
 }
 
-// Token tile u of the guided step: accumulator 0 = conditional rows, accumulator 1 = the
-// unconditional rows of the same tokens (tb1 = tb0 + 128).  x[lat] += dt * (v_u + cfg (v_c - v_u))
-// with v = acc + bias, in the order and rounding of the standalone CFG + Euler kernel.
-__device__ __forceinline__ void epi_out_cfg(const EpiParams& ep, uint32_t tb0, int tok, int half) {
+// The guided step's output projection, for one tile of 128 image tokens and one 64-column half nh of
+// the 128 patch features: accumulator 0 (TMEM columns 0..63) holds the conditional rows, accumulator
+// 1 (columns 64..127) the unconditional rows of the same tokens; warp half h takes the 32 features
+// of chunk c = 2 nh + h (dy = nh, dx = h).  x[lat] += dt * (v_u + cfg (v_c - v_u)) with v = acc +
+// bias, in the order and rounding of the standalone CFG + Euler kernel.
+__device__ __forceinline__ void epi_out_cfg(const EpiParams& ep, uint32_t tb0, int tok, int nh, int half) {
   const bool valid = tok < ep.n_img;
   const int r = tok / ep.grid_w;
   const int cc = tok - r * ep.grid_w;
+  const int c = 2 * nh + half;
+  float vc[32], vu[32];
+  tmem_ld32f(tb0 + half * 32, vc);
+  tmem_ld32f(tb0 + 64 + half * 32, vu);
+  if (valid) {
+    const int dy = c >> 1, dx = c & 1;
+    float4* xp = reinterpret_cast<float4*>(ep.x_lat +
+                                           ((static_cast<int64_t>(2 * r + dy) * ep.lat_w8) + 2 * cc + dx) * 32);
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int c = half * 2 + q;
-    float vc[32], vu[32];
-    tmem_ld32f(tb0 + c * 32, vc);
-    tmem_ld32f(tb0 + 128 + c * 32, vu);
-    if (valid) {
-      const int dy = c >> 1, dx = c & 1;
-      float4* xp = reinterpret_cast<float4*>(
-          ep.x_lat + ((static_cast<int64_t>(2 * r + dy) * ep.lat_w8) + 2 * cc + dx) * 32);
+    for (int i = 0; i < 8; ++i) {
+      float4 a = xp[i];
+      float cv[4], uv[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float4 a = xp[i];
-        float cv[4], uv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float bj = __bfloat162float(ep.bias[c * 32 + 4 * i + e]);
-          cv[e] = vc[4 * i + e] + bj;
-          uv[e] = vu[4 * i + e] + bj;
-        }
-        a.x = fmaf(ep.dt, fmaf(ep.cfg, cv[0] - uv[0], uv[0]), a.x);
-        a.y = fmaf(ep.dt, fmaf(ep.cfg, cv[1] - uv[1], uv[1]), a.y);
-        a.z = fmaf(ep.dt, fmaf(ep.cfg, cv[2] - uv[2], uv[2]), a.z);
-        a.w = fmaf(ep.dt, fmaf(ep.cfg, cv[3] - uv[3], uv[3]), a.w);
-        xp[i] = a;
+      for (int e = 0; e < 4; ++e) {
+        const float bj = __bfloat162float(ep.bias[c * 32 + 4 * i + e]);
+        cv[e] = vc[4 * i + e] + bj;
+        uv[e] = vu[4 * i + e] + bj;
       }
+      a.x = fmaf(ep.dt, fmaf(ep.cfg, cv[0] - uv[0], uv[0]), a.x);
+      a.y = fmaf(ep.dt, fmaf(ep.cfg, cv[1] - uv[1], uv[1]), a.y);
+      a.z = fmaf(ep.dt, fmaf(ep.cfg, cv[2] - uv[2], uv[2]), a.z);
+      a.w = fmaf(ep.dt, fmaf(ep.cfg, cv[3] - uv[3], uv[3]), a.w);
+      xp[i] = a;
     }
   }
 }
@@ -373,7 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kPer = EPI == kEpiOutCfg ? 2 : 1;
   const int num_m = (ep.M + kBM - 1) / kBM;
   const int num_n = (ep.N + BN - 1) / BN;
-  const int num_units = EPI == kEpiOutCfg ? (ep.n_img + kBM - 1) / kBM : num_m * num_n;
+  constexpr int kHalves = EPI == kEpiOutCfg ? 128 / BN : 1;  // N-parts of the 128 patch features
+  const int num_units = EPI == kEpiOutCfg ? ((ep.n_img + kBM - 1) / kBM) * kHalves : num_m * num_n;
   const int num_kb = ep.K / kBK;
 
   if (threadIdx.x == 0) {
@@ -414,8 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int sub = 0; sub < kPer && ok; ++sub) {
           int arow, brow;
           if constexpr (EPI == kEpiOutCfg) {
-            arow = sub * ep.n_img + unit * kBM;  // branch `sub`, tokens unit*128 ..
-            brow = 0;
+            arow = sub * ep.n_img + (unit / kHalves) * kBM;  // branch `sub`, tokens (unit / kHalves) * 128 ..
+            brow = (unit % kHalves) * BN;
           } else {
             int mb, nb;
             tile_coords(unit, num_m, num_n, mb, nb);
@@ -506,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: TMEM loads are .sync.aligned
         tc_fence_after();
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-        epi_out_cfg(ep, tb, unit * kBM + quad * 32 + lane, half);
+        epi_out_cfg(ep, tb, (unit / kHalves) * kBM + quad * 32 + lane, unit % kHalves, half);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -755,7 +757,7 @@ cudaError_t launch_single(const CUtensorMap& a, const CUtensorMap& b, const EpiP
     if (e != cudaSuccess) return e;
     mark_configured_on_device(configured);
   }
-  const int tiles = EPI == kEpiOutCfg ? (ep.n_img + kBM - 1) / kBM
+  const int tiles = EPI == kEpiOutCfg ? ((ep.n_img + kBM - 1) / kBM) * (128 / BN)
                                      : ((ep.M + kBM - 1) / kBM) * ((ep.N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (grid <= 0) return cudaSuccess;
@@ -801,7 +803,7 @@ cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& a, const CUtensorMap& b
     case kEpiSwiglu: return launch_pair<kEpiSwiglu>(a, b, b2, ep, s, err);
     case kEpiEmbed: return launch_pair<kEpiEmbed>(a, b, b2, ep, s, err);
     case kEpiOut: return launch_single<128, kEpiOut>(a, b, ep, s, err);
-    case kEpiOutCfg: return launch_single<128, kEpiOutCfg>(a, b, ep, s, err);
+    case kEpiOutCfg: return launch_single<64, kEpiOutCfg>(a, b, ep, s, err);  // b: box of 64 rows
   }
   return cudaErrorInvalidValue;
 }

@@ -84,7 +84,7 @@ void count_launches(int n);
 
 // ------------------------------------------------------------------ kernels
 // Every GEMM tensor map (A = activations [M, K], B = weights [N, K], BF16) has the box
-// {kGemmBoxK, kGemmBoxRows}: the kernels' shared-memory layout and transaction counts are
+// {kGemmBoxK, kGemmBoxRows} (the guided output projection: B with 64-row boxes): the kernels' shared-memory layout and transaction counts are
 // derived from these two constants.  For kEpiSwiglu, b = gate rows and b2 = up rows.
 constexpr uint32_t kGemmBoxK = 64;
 constexpr uint32_t kGemmBoxRows = 128;

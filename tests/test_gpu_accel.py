@@ -17,7 +17,7 @@ import torch
 import diffusion_transformer_text_block_b200 as moss
 
 import oracle.moss_oracle as o
-from tests.gpu_common import assert_no_device_error, make_model, psnr
+from tests.gpu_common import assert_no_device_error, make_model, psnr, rel_l2
 from synth import TINY, make_text
 
 pytestmark = pytest.mark.gpu
@@ -133,10 +133,13 @@ def test_three_pass_slg_matches_oracle(n_u):
     tc = make_text(1, 16, TINY.hidden, 102)[0]
     tu = make_text(1, max(n_u, 1), TINY.hidden, 103)[0][:n_u].contiguous()
     out, _, _ = _gpu(model, tc, tu, steps, slg_scale=2.0)
+    out_two, _, _ = _gpu(model, tc, tu, steps)
     ref, _, _ = _oracle(wn, tc, tu, steps, slg_scale=2.0)
     two, _, _ = _oracle(wn, tc, tu, steps)
     assert psnr(ref, out) >= 40.0
-    assert psnr(ref, two) < psnr(ref, out)          # the third pass does change the result
+    # The third pass changes the result, on both sides.  (Its effect on this 2-layer model can be as
+    # small as the GPU path's BF16 rounding, so the two are not compared with each other.)
+    assert rel_l2(two, ref) > 1e-5 and rel_l2(out_two, out) > 1e-5
     model.close()
     assert_no_device_error()
 
