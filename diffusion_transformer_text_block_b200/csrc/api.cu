@@ -399,11 +399,16 @@ struct LayerRes {
   const float* k_gain;
 };
 
-// M-tiles per band of the pair GEMMs' tile order, per GEMM of the block, chosen by DRAM bytes per
-// launch at the 1024^2 shape (M = 9216, 36 pair tiles along M) with equal launch times: down (K =
-// 8192) reads 639 MB with bands of 4 against 751 MB with 16 (its 4 MB activation band per M-tile
-// stays in L2 across the N-tiles), O-proj 199 against 218 MB with 8, QKV and gate/up least with 16.
-constexpr int kBandQkv = 16, kBandOproj = 8, kBandGateUp = 16, kBandDown = 4;
+// M-tiles per band of the pair GEMMs' tile order and L2 eviction hints of their A and B loads (0
+// none, 1 evict first, 2 evict last), per GEMM of the block, chosen by DRAM bytes per launch at the
+// 1024^2 shape (M = 9216, 36 pair tiles along M), all with equal launch times.  Down (K = 8192)
+// visits all N-tiles of one M-tile before the next, streams its activations (evict first) and keeps
+// its 50 MB of weights (evict last): 567 MB read against 751 MB with bands of 16 and no hints.
+// O-proj: bands of 8, weights kept (190 against 218 MB).  QKV and gate/up read least with bands of
+// 16 and no hints (hints or whole-M bands raised QKV from 237 to 343-436 MB and gate/up from 362 to
+// 433-680 MB).
+constexpr int kBandQkv = 16, kBandOproj = 8, kBandGateUp = 16, kBandDown = 1;
+constexpr int kL2Qkv[2] = {0, 0}, kL2Oproj[2] = {0, 2}, kL2GateUp[2] = {0, 0}, kL2Down[2] = {1, 2};
 
 int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<int>& lens, const float* mod_l,
                  cudaStream_t s) {
@@ -435,6 +440,8 @@ int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<
   q.split_rows = equal ? 0 : static_cast<int>(M - lens[nb - 1]);
   q.rope_stride = m->rope_n;
   q.group_m = kBandQkv;
+  q.a_l2 = kL2Qkv[0];
+  q.b_l2 = kL2Qkv[1];
   LAUNCH(m, MOSS_K_GEMM_QKV, s, launch_gemm(kEpiQkv, tm_h, *lw.qkv, *lw.qkv, q, s, m->err), "qkv gemm");
 
   if (equal) {
@@ -454,6 +461,8 @@ int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<
   o.M = M; o.N = D; o.K = D;
   o.out_f32 = x; o.gate = mod_l + 2 * D;
   o.group_m = kBandOproj;
+  o.a_l2 = kL2Oproj[0];
+  o.b_l2 = kL2Oproj[1];
   LAUNCH(m, MOSS_K_GEMM_OPROJ, s, launch_gemm(kEpiResid, tm_attn, *lw.wo, *lw.wo, o, s, m->err),
          "out-projection gemm");
 
@@ -464,6 +473,8 @@ int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<
   g.M = M; g.N = F; g.K = D;
   g.out_bf16 = m->act;
   g.group_m = kBandGateUp;
+  g.a_l2 = kL2GateUp[0];
+  g.b_l2 = kL2GateUp[1];
   LAUNCH(m, MOSS_K_GEMM_GATEUP, s, launch_gemm(kEpiSwiglu, tm_h, *lw.wg, *lw.wu, g, s, m->err),
          "gate/up gemm");
 
@@ -471,6 +482,8 @@ int block_impl_w(moss_model* m, const LayerRes& lw, float* x, const std::vector<
   d.M = M; d.N = D; d.K = F;
   d.out_f32 = x; d.gate = mod_l + 5 * D;
   d.group_m = kBandDown;
+  d.a_l2 = kL2Down[0];
+  d.b_l2 = kL2Down[1];
   LAUNCH(m, MOSS_K_GEMM_DOWN, s, launch_gemm(kEpiResid, tm_act, *lw.wd, *lw.wd, d, s, m->err),
          "down gemm");
   return MOSS_OK;

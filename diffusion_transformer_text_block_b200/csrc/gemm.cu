@@ -621,6 +621,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int s2 = 0; s2 < S::kStages; ++s2) armed[s2] = -1;
       const CUtensorMap* bmap = (EPI == kEpiSwiglu && !leader) ? &tmB2 : &tmB;
+      const uint64_t a_pol = l2_policy(ep.a_l2), b_pol = l2_policy(ep.b_l2);
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         int mb, nb;
         tile_coords(tile, num_m, num_n, mb, nb, group_m);
@@ -637,8 +638,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             armed[stage] = static_cast<int>(phase);
             mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
           }
-          tma_load_2d_pair(sA + stage * S::kABytes, &tmA, full_leader, kb * kBK, arow);
-          tma_load_2d_pair(sB + stage * S::kBBytes, bmap, full_leader, kb * kBK, brow);
+          if (ep.a_l2)
+            tma_load_2d_pair_hint(sA + stage * S::kABytes, &tmA, full_leader, kb * kBK, arow, a_pol);
+          else
+            tma_load_2d_pair(sA + stage * S::kABytes, &tmA, full_leader, kb * kBK, arow);
+          if (ep.b_l2)
+            tma_load_2d_pair_hint(sB + stage * S::kBBytes, bmap, full_leader, kb * kBK, brow, b_pol);
+          else
+            tma_load_2d_pair(sB + stage * S::kBBytes, bmap, full_leader, kb * kBK, brow);
           if (++stage == S::kStages) {
             stage = 0;
             phase ^= 1;

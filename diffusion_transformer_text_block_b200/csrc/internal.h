@@ -63,6 +63,8 @@ struct EpiParams {
   float eps = 1e-6f;
   int group_m = 16;                  // pair GEMMs: M-tiles per band of the tile order (all N-tiles of
                                      // a band before the next band)
+  int a_l2 = 0, b_l2 = 0;            // pair GEMMs: L2 eviction hint of the A and B loads (0 none,
+                                     // 1 evict first, 2 evict last)
 };
 
 // ------------------------------------------------------------------ tensor maps
