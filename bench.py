@@ -202,6 +202,10 @@ def cpu_baseline(run_once=None):
                       f"forwards/s = 1/(42 x block time)"}
 
 
+REFERENCE_SAMPLE = ("one branch-block of the 1024^2 workload per timed step (4608 tokens x hidden 3072, "
+                    "float64 oracle), extrapolated to the step's 83 branch-blocks")
+
+
 def run_reference(args):
     """The oracle as it stands, on the host cores: each of the --steps timed steps runs one
     branch-block of the workload (a bounded sample of the step's 83), and the step time is

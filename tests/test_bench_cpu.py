@@ -83,3 +83,18 @@ def test_committed_traffic_records_are_well_formed():
         assert rec["dram_bytes_per_launch"] > 0
         assert all(os.path.exists(os.path.join(ROOT, f)) for f in rec["sources"])
         assert os.path.exists(os.path.join(ROOT, rec["summary"]))
+
+
+def test_reference_arm_line_names_its_extrapolation(capsys):
+    """bench.py --impl reference: the oracle on one branch-block per timed step, the JSON line says
+    that the step figure is extrapolated and what was timed."""
+    import argparse
+    import json
+
+    bench.run_reference(argparse.Namespace(steps=1, warmup=0, gpus=1))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["extrapolated"] is True
+    assert line["steps"] == 1 and line["warmup"] == 0
+    assert "branch-block" in line["timed_per_step"] and line["dtype"] == "f64"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]

@@ -139,6 +139,28 @@ def test_denoise_step_cfg1_and_sample_consistency():
     assert_no_device_error()
 
 
+def test_denoise_step_schedule_reuse_matches_per_step_modulation():
+    """moss_denoise_step computes a schedule's modulation once and reuses it (steps <= max_steps); with
+    steps > max_steps each call computes its own step's vectors.  Both give the same steps bit for bit,
+    also after a forward call in between has dropped the stored schedule."""
+    a, wg, _ = make_model(TINY, 79, max_tokens=32, max_latent_hw=64, max_steps=8)
+    b = moss.Model(TINY, wg, max_tokens=32, max_batch=2, max_latent_hw=64, max_steps=4)
+    tc = make_text(1, 16, TINY.hidden, 80)[0].cuda()
+    tu = make_text(1, 9, TINY.hidden, 81)[0].cuda()
+    x0 = make_latent(8, 8, 82).cuda()
+    xa, xb = x0.clone(), x0.clone()
+    for i in range(8):
+        a.denoise_step(xa, tc, tu, 64, 64, i, 8, uncond_skip_layers=[1])
+        b.denoise_step(xb, tc, tu, 64, 64, i, 8, uncond_skip_layers=[1])   # 8 > max_steps: per call
+        if i == 3:
+            a.forward(x0, torch.stack([tc, tc]), 64, 64, 0.5)              # drops the stored schedule
+    torch.cuda.synchronize()
+    assert torch.equal(xa, xb)
+    a.close()
+    b.close()
+    assert_no_device_error()
+
+
 def test_denoise_step_host_buffers_match_device_step():
     """moss_denoise_step_host (latent and prompts in host memory, pinned and pageable) gives the
     device-buffer step's result bit for bit, with a ragged negative prompt and at cfg 1."""
