@@ -107,6 +107,12 @@ def test_elementwise_entry_points_check_arguments_without_launching():
     assert lib.moss_selftest_attention_timeout(a16, b16, 1, 256, 1, -1, None) == 1
     assert lib.moss_selftest_attention_timeout(a16, b16, 1, 256, 1, 2, None) == 1          # 2 key steps
     assert lib.moss_selftest_attention_timeout(None, b16, 1, 256, 1, 0, None) == 1
+    # the host-buffer step: bad schedule arguments, a NULL model and NULL buffers are refused first
+    hx = (ctypes.c_float * 32)()
+    assert lib.moss_denoise_step_host(None, hx, hx, 1, hx, 1, 64, 64, 0, 0, 3.0, 5.0, None, 0, 0.01, 1.0, None) == 1
+    assert lib.moss_denoise_step_host(None, hx, hx, 1, hx, 1, 64, 64, 4, 4, 3.0, 5.0, None, 0, 0.01, 1.0, None) == 1
+    assert lib.moss_denoise_step_host(None, hx, hx, 1, hx, 1, 64, 64, 0, 4, 3.0, 5.0, None, 0, 0.01, 1.0, None) == 1
+    assert "model" in lib.moss_last_error().decode()
     assert lib.moss_launch_count(0) == before
 
 
