@@ -321,6 +321,30 @@ def test_full_guided_step_fused_update_matches_forward_and_update(full_model):
     assert_no_device_error()
 
 
+def test_guided_step_fused_update_with_more_tiles_than_sms():
+    """The fused update on a 2000 x 1936 image (125 x 121 = 15125 image tokens: 119 token tiles, the last
+    partial, so 238 work units over at most 148 CTAs, each CTA taking several): tiny model, a 16-token
+    prompt and a 3-token negative prompt; bit for bit against the two forwards and the standalone update."""
+    h, w = 2000, 1936
+    n_img = (h // 16) * (w // 16)
+    model, wg, wn = make_model(TINY, 151, max_tokens=n_img + 16, max_latent_hw=(h // 8) * (w // 8))
+    x0 = make_latent(h // 8, w // 8, 152).cuda()
+    tc = make_text(1, 16, TINY.hidden, 153)[0].cuda()
+    tu = make_text(1, 3, TINY.hidden, 154)[0].cuda()
+    x = x0.clone()
+    model.denoise_step(x, tc, tu, h, w, 2, 10, 3.0, 5.0, [1], 0.01, 1.0)
+    sig = o.sigma_schedule(10, 5.0)
+    vc = model.forward(x0, tc[None], h, w, float(sig[2]), skip_layers=[[]]).clone()
+    vu = model.forward(x0, tu[None], h, w, float(sig[2]), skip_layers=[[1]]).clone()
+    ref = x0.clone()
+    moss.cfg_euler_step(ref, vc[0].contiguous(), vu[0].contiguous(), 3.0, float(sig[2]), float(sig[3]))
+    torch.cuda.synchronize()
+    assert torch.equal(x, ref)
+    assert rel_l2(x.cpu().numpy(), x0.cpu().numpy()) > 1e-3
+    model.close()
+    assert_no_device_error()
+
+
 @pytest.mark.parametrize("n_u", [5, 0])
 def test_sample_tiny_short_negative_prompt(n_u):
     """Branches of different text lengths (n_u = 0: the empty negative prompt): the tiny
