@@ -26,6 +26,10 @@
  *     validated on the host before anything is launched; an invalid call launches nothing.
  *   - After MOSS_ERR_CUDA the model should be freed ([MI] C API rules: after a CUDA error,
  *     free the engine).
+ *   - A model holds mutable state: its workspace, the modulation of the last schedule it
+ *     computed, the host-step staging buffers.  Calls on one model must not overlap: use it from
+ *     one thread at a time and on one stream (or order the streams); separate models are
+ *     independent.
  *   - Floating-point layouts are row-major, innermost index last.
  *
  * Model tensors (D = hidden, H = heads, d = head_dim = 128, F = ffn, L = layers,
