@@ -321,6 +321,31 @@ def test_full_guided_step_fused_update_matches_forward_and_update(full_model):
     assert_no_device_error()
 
 
+def test_full_guided_step_2048_fused_update(full_model):
+    """The long-sequence stress shape (2048^2: 16384 image tokens, a 4096-token prompt -- the pages'
+    maximum -- and a 77-token negative prompt) with the full model: the guided step, whose fused update
+    runs 256 work units over at most 148 CTAs, equals the two branch forwards followed by the
+    standalone CFG + Euler kernel, bit for bit."""
+    from synth import FULL
+    _, w = full_model
+    model = moss.Model(FULL, w, max_tokens=16384 + 4096, max_batch=2, max_latent_hw=256 * 256, max_steps=10)
+    x0 = make_latent(256, 256, 27, device="cuda")
+    tc = make_text(1, 4096, FULL.hidden, 28, device="cuda")[0].contiguous()
+    tu = make_text(1, 77, FULL.hidden, 29, device="cuda")[0].contiguous()
+    x = x0.clone()
+    model.denoise_step(x, tc, tu, 2048, 2048, 1, 10, 3.0, 5.0, [22], 0.01, 1.0)
+    sig = o.sigma_schedule(10, 5.0)
+    vc = model.forward(x0, tc[None], 2048, 2048, float(sig[1]), skip_layers=[[]]).clone()
+    vu = model.forward(x0, tu[None], 2048, 2048, float(sig[1]), skip_layers=[[22]]).clone()
+    ref = x0.clone()
+    moss.cfg_euler_step(ref, vc[0].contiguous(), vu[0].contiguous(), 3.0, float(sig[1]), float(sig[2]))
+    torch.cuda.synchronize()
+    assert torch.equal(x, ref)
+    assert torch.isfinite(x).all() and rel_l2(x.cpu().numpy(), x0.cpu().numpy()) > 1e-3
+    model.close()
+    assert_no_device_error()
+
+
 def test_guided_step_fused_update_with_more_tiles_than_sms():
     """The fused update on a 2000 x 1936 image (125 x 121 = 15125 image tokens: 119 token tiles, the last
     partial, so 238 work units over at most 148 CTAs, each CTA taking several): tiny model, a 16-token
