@@ -59,3 +59,29 @@ def test_attention_wait_gives_up_and_every_warp_finishes():
     for _ in range(2):
         assert rel(moss.op_attention(qkv, H)) < 1e-2
         assert moss.device_status(clear=True) == 0
+
+
+def test_attention_wait_gives_up_in_a_grid_larger_than_the_gpu():
+    """192 CTAs, more than one wave: the CTA that loses a V tile gives up while the other CTAs,
+    and the later wave on the SMs they free, complete; the launch ends, the error word holds the
+    code, and later launches are correct."""
+    B, N, H = 2, 1024, 24
+    g = torch.Generator(device="cuda").manual_seed(5)
+    qkv = torch.randn(B, N, 3 * H * 128, generator=g, device="cuda").to(torch.bfloat16)
+    q, k, v = qkv.view(B, N, 3, H, 128).permute(2, 0, 3, 1, 4).float()
+    ref = F.scaled_dot_product_attention(q, k, v).permute(0, 2, 1, 3).reshape(B, N, H * 128)
+
+    def rel(o):
+        return ((o.float() - ref).norm() / ref.norm()).item()
+
+    assert moss.device_status(clear=True) == 0
+    assert rel(moss.op_attention(qkv, H)) < 1e-2
+    t0 = time.time()
+    moss.selftest_attention_timeout(qkv, H, 3)
+    status = moss.device_status(clear=True)  # synchronises
+    elapsed = time.time() - t0
+    assert status in (0x201, 0x202)
+    assert 1.0 < elapsed < 60.0
+    for _ in range(2):
+        assert rel(moss.op_attention(qkv, H)) < 1e-2
+        assert moss.device_status(clear=True) == 0

@@ -40,10 +40,14 @@ def test_gemm_bf16(M, N, K):
 
 @pytest.mark.parametrize("B,N,H,qscale", [(1, 32, 2, 1.0), (2, 200, 2, 1.0), (2, 384, 3, 1.0), (1, 520, 2, 4.0),
                                           (2, 1, 1, 1.0), (1, 300, 1, 32.0), (1, 129, 1, 1.0), (1, 255, 1, 1.0),
-                                          (2, 257, 1, 1.0), (1, 511, 2, 1.0)])
+                                          (2, 257, 1, 1.0), (1, 511, 2, 1.0),
+                                          (2, 100, 80, 1.0), (2, 520, 64, 1.0), (2, 1100, 24, 1.0)])
 def test_attention(B, N, H, qscale):
     """Against the oracle; qscale 32 spreads a row's scores over several hundred (log2 units), so
-    exponent arguments fall below -126, where the kernel's polynomial exponentials clamp."""
+    exponent arguments fall below -126, where the kernel's polynomial exponentials clamp.
+    The last three shapes launch more CTAs (256-query block, head, branch) than the GPU has SMs:
+    one key step per CTA with 80 heads, a ragged key tail of 8 with 64 heads, and a last query
+    block of 76 rows (its tile B entirely past the sequence end) with 24 heads."""
     D = H * 128
     q = _bf16((B, N, D), 3, qscale)
     k = _bf16((B, N, D), 4)
